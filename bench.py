@@ -1,0 +1,545 @@
+#!/usr/bin/env python
+"""Throughput of the TriAttention key-importance + eviction step on B200.
+
+One step = tri_compress_step over one synthetic cache: effective query,
+score of every cached key, top-B selection with a recent window, and
+forward-packing compaction of the kept K/V rows.  Default workload: 32
+layers x 8 KV heads, GQA group 4, one sequence of 32768 cached bf16 keys,
+RoPE base 5e5, offsets 1..4096, B = 2048, W = 128.
+
+Metric: cached keys scored+selected+compacted per second (whole job, all
+ranks), with the achieved HBM GB/s of the dominant (score) kernel and of the
+whole step against the measured B200 copy bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU)
+
+Timing: each timed step restores the kept region of the cache and flushes L2
+(256 MiB write) outside CUDA events that bracket only the tri_compress_step
+launches; the K/V pools (4.3 GB) are larger than L2 as well.  The timed loop
+is bracketed by a barrier and a device synchronize; the step time is the
+maximum over ranks.  Ranks run independent caches (weak scaling: units
+shard across GPUs with no data-path collective).
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "cached keys scored+selected+compacted per sec; achieved HBM GB/s vs peak"
+UNIT = "keys/s"
+FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 7700.0
+L2_FLUSH_BYTES = 256 << 20
+SCORE_SOURCES = ["score.cu", "tri_device.cuh", "tri_internal.h"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="cfg2", help="cfg1 | cfg2 | cfg4 | cfg5")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def score_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in SCORE_SOURCES:
+        with open(os.path.join(ROOT, "rope_aware_kv_tri_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic_per_key():
+    """DRAM bytes per scored key of the score kernel from the committed ncu
+    summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "score_kernel_traffic.txt")
+    try:
+        kv = {}
+        with open(path) as f:
+            for line in f:
+                if "=" in line and not line.lstrip().startswith("#"):
+                    k, v = line.split("=", 1)
+                    kv[k.strip()] = v.strip()
+        if kv.get("source_sha256") != score_source_hash():
+            return None
+        return float(kv["dram_bytes_per_key"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+        self.bus = None
+        try:
+            import torch
+            self.bus = int(torch.cuda.get_device_properties(device_index).pci_bus_id)
+        except Exception:
+            pass
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu=pci.bus_id,{self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.5)
+        self.t0 = time.time()
+
+    def stop(self):
+        self.t1 = time.time()
+        time.sleep(0.3)
+        if self.proc is None:
+            return
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            try:
+                bus = int(f[0].split(":")[1], 16)
+            except Exception:
+                bus = None
+            if self.bus is not None and bus is not None and bus != self.bus:
+                continue
+            f = f[1:]
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except Exception:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        if args.impl == "reference":
+            return world, rank, local, None
+        import torch
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+        return world, rank, local, dist
+    return world, rank, local, None
+
+
+def unit_rows(pool, table_row, length, l, h):
+    """Rows [0, length) of (layer l, KV head h) of one sequence of a paged pool."""
+    import torch
+    nb = -(-length // 16)
+    blocks = torch.tensor(table_row[:nb], dtype=torch.long, device=pool.device)
+    return pool[l, blocks, h].reshape(nb * 16, pool.shape[-1])[:length]
+
+
+# ---------------------------------------------------------- oracle sample
+
+def oracle_sample(units, stats_fn, deltas, base, budget, window, seconds):
+    """Time the float64 oracle on units until about ``seconds`` have passed.
+
+    ``units`` yields (keys_bf16_cpu [T,128], vals_bf16_cpu, (s, l, h), p).
+    Returns (keys scored, seconds, units done).
+    """
+    import numpy as np
+    import torch
+    import oracle
+    try:
+        from threadpoolctl import threadpool_limits
+        limit = threadpool_limits(1)
+    except Exception:
+        limit = None
+    keys_done, t_used, n = 0, 0.0, 0
+    for keys, vals, (s, l, h), p in units:
+        qb, qa, r = stats_fn(l, h)
+        kf = keys.double().numpy()
+        kb, vb = keys.view(torch.int16).numpy(), vals.view(torch.int16).numpy()
+        t0 = time.perf_counter()
+        oracle.compress_unit(kf, kb, vb, qb, qa, r, p, deltas, base, budget, window)
+        t_used += time.perf_counter() - t0
+        keys_done += kf.shape[0]
+        n += 1
+        if t_used >= seconds:
+            break
+    if limit is not None:
+        limit.restore_original_limits()
+    return keys_done, t_used, n
+
+
+# --------------------------------------------------------------- our arm
+
+def run_ours(args, world, rank, local, dist):
+    import numpy as np
+    import torch
+    import rope_aware_kv_tri_b200 as tri
+    from rope_aware_kv_tri_b200 import build_lib
+    from workload import CONFIGS, make_workload
+
+    build_lib.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    cfg = CONFIGS[args.workload]
+    if args.workload == "cfg3":
+        raise SystemExit("the decode-loop workload is measured by tests/test_gpu_workloads.py, not here")
+    wl = make_workload(cfg, device=dev, seed=rank)
+    L, Hkv, G, Hq, S = cfg.L, cfg.Hkv, cfg.G, cfg.Hq, cfg.S
+    B, W = cfg.budget, cfg.window
+    stream = torch.cuda.current_stream(dev)
+
+    # statistics: one-time calibration on the device (untimed)
+    if wl.qbar is not None:
+        qbar, qabs, R = wl.qbar, wl.qabs, wl.R
+    else:
+        qbar = torch.empty(L, Hq, 128, device=dev)
+        qabs = torch.empty(L, Hq, 64, device=dev)
+        R = torch.empty(L, Hq, device=dev)
+        tri.tri_calibrate_centers(wl.q_samples, qbar, qabs, R)
+        torch.cuda.synchronize(dev)
+
+    lens = wl.seq_len.cpu().tolist()
+    kept_blocks = [min((n + 15) // 16, (B + 15) // 16) for n in lens]
+    keys_per_step = sum(lens) * L * Hkv
+    cache = tri.KvCache(wl.k_pool, wl.v_pool, wl.block_table, wl.seq_len, wl.cur_pos,
+                        torch.zeros(1, dtype=torch.int32, device=dev), G)
+    ws = tri.alloc_workspace(cache, B)
+    freed = torch.empty(S * wl.max_blocks, dtype=torch.int32, device=dev)
+    count = torch.empty(1, dtype=torch.int32, device=dev)
+
+    # the rows a step may rewrite: blocks holding slots [0, B) of each sequence
+    rblocks = torch.cat([wl.block_table[s, :kept_blocks[s]].long() for s in range(S)])
+    save_k = wl.k_pool[:, rblocks].clone()
+    save_v = wl.v_pool[:, rblocks].clone()
+    save_len = wl.seq_len.clone()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def restore():
+        wl.k_pool[:, rblocks] = save_k
+        wl.v_pool[:, rblocks] = save_v
+        wl.seq_len.copy_(save_len)
+        flush.zero_()
+
+    def step(events=None, idx_out=None):
+        tri.tri_compress_step(cache, qbar, qabs, R, cfg.base, wl.deltas, B, W, freed, count, ws,
+                              idx_out=idx_out, events=events)
+
+    # census (untimed): how many rows a step moves, from its kept indices
+    idx = torch.empty(S, L, Hkv, B, dtype=torch.int32, device=dev)
+    restore()
+    step(idx_out=idx)
+    if tri.tri_sync_status(cache.status) != tri.TRI_OK:
+        raise RuntimeError("device status flag raised by the census step")
+    moved = 0
+    for s in range(S):
+        if lens[s] > B:
+            j = torch.arange(B, device=dev, dtype=torch.int32)
+            moved += int((idx[s] != j).sum().item())
+    del idx
+    freed_per_step = int(count.item())
+
+    for _ in range(args.warmup):
+        restore()
+        step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    for k in range(args.steps):
+        restore()
+        step(events=evs[k])
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    clocks.stop()
+    if tri.tri_sync_status(cache.status) != tri.TRI_OK:
+        raise RuntimeError("device status flag raised during the timed steps")
+
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    query_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    score_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    evict_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * keys_per_step * args.steps / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    peak, peak_kind = measured_peak()
+    k_bytes = keys_per_step * 256
+    moved_bytes = moved * 4 * 256
+    score_mean = statistics.mean(score_ms)
+    achieved = k_bytes / (score_mean / 1e3) / 1e9
+    tpk = recorded_traffic_per_key()
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                "frac": round(achieved / peak, 4), "traffic": (round(tpk * keys_per_step) if tpk else None),
+                "kernel": "score_kernel", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_kind == "measured" else "fallback 6650 GB/s",
+                "algorithmic_bytes_per_launch": k_bytes, "ms_per_launch": round(score_mean, 5),
+                "nominal_hbm_gbs": NOMINAL_HBM_GBS}
+    step_bytes = k_bytes + moved_bytes
+    step_achieved = step_bytes / (ms_per_step / 1e3) / 1e9
+    step_roofline = {"bound": "hbm", "achieved": round(step_achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(step_achieved / peak, 4), "bytes_per_step": step_bytes,
+                     "moved_rows": moved, "phase_ms": {"query": round(statistics.mean(query_ms), 5),
+                                                       "score": round(score_mean, 5),
+                                                       "select_compact": round(statistics.mean(evict_ms), 5)}}
+
+    # ------------------------------------------------------------ e2e
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, tri, cache, wl, cfg, qbar, qabs, R, ws, freed, count, save_k, save_v, rblocks,
+                      save_len, keys_per_step, dev, world, dist)
+
+    # ---------------------------------------------------- cpu baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens)
+
+    clk = clocks.summary()
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "seq_lens": lens,
+                   "budget": B, "window": W, "rope_base": cfg.base, "deltas": wl.deltas,
+                   "keys_per_step_per_gpu": keys_per_step, "freed_blocks_per_step": freed_per_step,
+                   "parallelism": f"units sharded: one independent cache per GPU x{world}",
+                   "input_dtype": "bf16 K/V, fp32 arithmetic",
+                   "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
+                   "timing": "CUDA events around each tri_compress_step; kept-region restore untimed"},
+        "roofline": roofline, "step_roofline": step_roofline,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_e2e(args, tri, cache, wl, cfg, qbar, qabs, R, ws, freed, count, save_k, save_v, rblocks, save_len,
+            keys_per_step, dev, world, dist):
+    """Same step through the C ABI with the cache in pinned HOST memory: the
+    timed region copies the inputs in, runs the step, and copies the result
+    (the kept region of K/V, new lengths, freed ids and count) back."""
+    import torch
+    wl.k_pool[:, rblocks] = save_k
+    wl.v_pool[:, rblocks] = save_v
+    wl.seq_len.copy_(save_len)
+    host = {n: t.to("cpu").pin_memory() for n, t in
+            (("k", wl.k_pool), ("v", wl.v_pool), ("table", wl.block_table), ("len", save_len),
+             ("pos", wl.cur_pos), ("qbar", qbar), ("qabs", qabs), ("R", R))}
+    out_k = torch.empty_like(save_k, device="cpu").pin_memory()
+    out_v = torch.empty_like(save_v, device="cpu").pin_memory()
+    out_len = torch.empty_like(save_len, device="cpu").pin_memory()
+    out_freed = torch.empty_like(freed, device="cpu").pin_memory()
+    out_count = torch.empty(1, dtype=torch.int32).pin_memory()
+    dev_in = {"k": wl.k_pool, "v": wl.v_pool, "table": wl.block_table, "len": wl.seq_len, "pos": wl.cur_pos,
+              "qbar": qbar, "qabs": qabs, "R": R}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in (out_k, out_v, out_len, out_freed, out_count))
+    times = []
+    for k in range(args.e2e_steps + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record()
+        for n, t in host.items():
+            dev_in[n].copy_(t, non_blocking=True)
+        tri.tri_compress_step(cache, qbar, qabs, R, cfg.base, wl.deltas, cfg.budget, cfg.window, freed, count, ws)
+        out_k.copy_(wl.k_pool[:, rblocks], non_blocking=True)
+        out_v.copy_(wl.v_pool[:, rblocks], non_blocking=True)
+        out_len.copy_(wl.seq_len, non_blocking=True)
+        out_freed.copy_(freed, non_blocking=True)
+        out_count.copy_(count, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize(dev)
+        if k > 0:                      # first call is a warm-up
+            times.append(a.elapsed_time(b))
+    if tri.tri_sync_status(cache.status) != tri.TRI_OK:
+        raise RuntimeError("device status flag raised during the end-to-end steps")
+    total = sum(times)
+    if dist is not None:
+        t = torch.tensor([total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    del host
+    return {"value": round(world * keys_per_step * len(times) / (total / 1e3), 1), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": len(times),
+            "ms_per_step": round(total / len(times), 3)}
+
+
+def run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens):
+    """The float64 oracle on a bounded sample of this workload's units, on
+    one host core (restored, untouched inputs)."""
+    import numpy as np
+    import torch
+    import oracle
+    wl.k_pool[:, rblocks] = save_k
+    wl.v_pool[:, rblocks] = save_v
+    table = wl.block_table.cpu().tolist()
+    rng = np.random.default_rng(1)
+    G = cfg.G
+    calib = {}
+
+    def stats_fn(l, h):
+        if (l, h) not in calib:
+            if wl.q_samples is not None:
+                calib[(l, h)] = oracle.calibrate(wl.q_samples[:, l, h * G:(h + 1) * G].double().cpu().numpy())
+            else:
+                sl = slice(h * G, (h + 1) * G)
+                calib[(l, h)] = tuple(t[l, sl].double().cpu().numpy() for t in (wl.qbar, wl.qabs, wl.R))
+        return calib[(l, h)]
+
+    def units():
+        while True:
+            s = int(rng.integers(cfg.S))
+            l = int(rng.integers(cfg.L))
+            h = int(rng.integers(cfg.Hkv))
+            n = lens[s]
+            yield (unit_rows(wl.k_pool, table[s], n, l, h).cpu(), unit_rows(wl.v_pool, table[s], n, l, h).cpu(),
+                   (s, l, h), int(wl.cur_pos[s].item()))
+
+    keys, secs, n = oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
+                                  args.cpu_seconds)
+    return {"value": round(keys / secs, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{n} random units of this workload ({keys} keys), float64 numpy oracle, 1 thread; "
+                      f"host has {os.cpu_count()} cores", "seconds": round(secs, 2)}
+
+
+# ---------------------------------------------------------- reference arm
+
+def run_reference(args, world, rank):
+    """The float64 CPU oracle as the reference arm (no GPU use)."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+    import oracle
+    from workload import CONFIGS, make_workload
+    cfg = CONFIGS[args.workload]
+    # The same per-unit shape and distributions as the full workload, one
+    # layer of it generated on the host.
+    small = cfg.replace(L=1, n_samples=min(cfg.n_samples, 1024))
+    wl = make_workload(small, device="cpu", seed=0)
+    G = cfg.G
+    if wl.qbar is not None:
+        stats = tuple(t.double().numpy() for t in (wl.qbar, wl.qabs, wl.R))
+    else:
+        stats = oracle.calibrate(wl.q_samples.double().numpy())
+    table = wl.block_table.tolist()
+    lens = wl.seq_len.tolist()
+    per_step = max(args.cpu_seconds / max(args.steps + args.warmup, 1), 0.5)
+
+    def units():
+        h = 0
+        while True:
+            s = h % cfg.S
+            hh = h % cfg.Hkv
+            n = lens[s]
+            k = oracle.unit_rows(wl.k_pool.view(torch.int16).numpy(), table[s], n, 0, hh)
+            v = oracle.unit_rows(wl.v_pool.view(torch.int16).numpy(), table[s], n, 0, hh)
+            yield (torch.from_numpy(k).view(torch.bfloat16), torch.from_numpy(v).view(torch.bfloat16),
+                   (s, 0, hh), int(wl.cur_pos[s]))
+            h += 1
+
+    def stats_fn(l, h):
+        return stats[0][0, h * G:(h + 1) * G], stats[1][0, h * G:(h + 1) * G], stats[2][0, h * G:(h + 1) * G]
+
+    it = units()
+    for _ in range(args.warmup):
+        oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, 0.0)
+    keys = secs = 0.0
+    n_units = 0
+    for _ in range(args.steps):
+        k, s_, n = oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, per_step)
+        keys += k
+        secs += s_
+        n_units += n
+    value = keys / secs
+    sample = (f"{n_units} units of the {cfg.name} workload shape over {args.steps} steps, float64 numpy "
+              f"oracle, 1 thread; host has {os.cpu_count()} cores")
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": cfg.name, "L": cfg.L, "Hkv": cfg.Hkv, "G": cfg.G, "D": 128,
+                      "seq_lens": cfg.lens, "budget": cfg.budget, "window": cfg.window},
+           "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+                            "sample": sample},
+           "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local, dist = dist_setup(args)
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+        return
+    try:
+        run_ours(args, world, rank, local, dist)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

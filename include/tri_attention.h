@@ -1,0 +1,254 @@
+/*
+ * tri_attention.h - C ABI of the B200 (sm_100a) TriAttention key-importance
+ * and eviction path.
+ *
+ * The library scores every cached post-rotary key of every (sequence, layer,
+ * KV head) unit from calibrated pre-rotary query statistics, keeps the
+ * top-B keys of each unit together with a recent window, and packs the kept
+ * K/V rows forward inside the sequence's paged blocks so that whole blocks
+ * become empty and can be returned to the caller's allocator.
+ *
+ * Pages cited (title, then section):
+ *   [Digest]   "TriAttention: Trigonometric KV Compression for Efficient Long
+ *               Reasoning" - "Core Mechanism", "Key Concepts"
+ *   [Abstract] "TriAttention: Efficient Long Reasoning with Trigonometric KV
+ *               Compression" - "English"
+ *   [GeoTrick] "TriAttention: How a Geometric Trick Cuts LLM Memory Use by 10x
+ *               Without Losing Accuracy" - "The Core Idea: Q/K Concentration
+ *               in Pre-RoPE Space", "Solving the Memory Fragmentation
+ *               Problem", "Why Existing KV Cache Compression Breaks in
+ *               Production"
+ *
+ * Notation: D = 128 (head dimension), n = D/2 = 64 rotary bands; band i pairs
+ * dimensions (i, i+64) (rotate-half) and turns by theta_i * position with
+ * theta_i = base^(-2i/D).  Query head hq = h*G + g belongs to KV head h.
+ *
+ * Conventions shared by every entry point:
+ *  - All array pointers are DEVICE memory owned by the caller, except where an
+ *    argument says "host".  The library allocates no device memory: scratch
+ *    comes from a caller-provided workspace sized by tri_workspace_size().
+ *  - Every call is asynchronous on the cudaStream_t it is given (0 = the
+ *    legacy default stream).  Host-side argument checks run before any
+ *    launch; a rejected call launches nothing and changes nothing.
+ *  - Errors a kernel can only see on the device (a block id out of range, a
+ *    sequence length larger than its table, a NaN score, a bounded wait that
+ *    gave up) are OR-ed as TRI_DEVFLAG_* bits into the caller's device status
+ *    word (tri_kv_desc.status).  tri_sync_status() reads and clears it.
+ *    After a device error the cache contents of the affected sequences are
+ *    unspecified; nothing outside the arrays named in the call is touched.
+ *  - Return value: TRI_OK, or the first error the host detected.
+ *  - Calls that share a descriptor, workspace or output buffers must not run
+ *    concurrently on different streams.
+ */
+#ifndef TRI_ATTENTION_H
+#define TRI_ATTENTION_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int tri_status;
+
+#define TRI_OK                 0
+#define TRI_ERR_INVALID        1  /* argument rejected on the host            */
+#define TRI_ERR_UNSUPPORTED    2  /* valid, but outside this build (D != 128) */
+#define TRI_ERR_CUDA           3  /* a CUDA runtime call or launch failed     */
+#define TRI_ERR_DEVICE_BOUNDS  4  /* device saw an out-of-range id or length  */
+#define TRI_ERR_TIMEOUT        5  /* a bounded device wait gave up            */
+#define TRI_ERR_NONFINITE      6  /* a NaN score was seen                     */
+#define TRI_ERR_WORKSPACE      7  /* workspace missing, small or misaligned   */
+
+/* Bits of the device status word. */
+#define TRI_DEVFLAG_BOUNDS     1
+#define TRI_DEVFLAG_TIMEOUT    2
+#define TRI_DEVFLAG_NONFINITE  4
+
+#define TRI_HEAD_DIM        128
+#define TRI_BLOCK_SIZE      16
+#define TRI_MAX_DELTAS      64
+#define TRI_MAX_BUDGET      16384
+
+/*
+ * The paged KV cache ([GeoTrick] "Why Existing KV Cache Compression Breaks
+ * in Production": fixed-size physical blocks handed out by a paged
+ * allocator).
+ *
+ *   k_pool, v_pool : bf16 [L][num_blocks][Hkv][block_size][D], 16-byte
+ *                    aligned; one (block, head) tile of 16 rows x 128 is
+ *                    4 KiB and contiguous.  Post-rotary keys; values.
+ *   block_table    : int32 [S][max_blocks]; entry b of sequence s is the pool
+ *                    block holding its slots 16b .. 16b+15, for every layer
+ *                    and head.  Only the first ceil(seq_len[s]/16) entries
+ *                    are read; each must lie in [0, num_blocks) and no block
+ *                    may appear twice among the entries in use.
+ *   seq_len        : int32 [S]; cached slots per (layer, head) of each
+ *                    sequence, in [0, max_blocks*16].  Compaction rewrites it.
+ *   cur_pos        : int64 [S]; position p of each sequence's next query.
+ *   status         : int32 [1]; device status word (TRI_DEVFLAG_* bits).
+ *   L, Hkv, G      : layers, KV heads per layer, query heads per KV head.
+ *   D, block_size  : must be 128 and 16 (TRI_ERR_UNSUPPORTED otherwise).
+ */
+typedef struct {
+    int L, Hkv, G, D, block_size;
+    void *k_pool;
+    void *v_pool;
+    int num_blocks;
+    const int32_t *block_table;
+    int S, max_blocks;
+    int32_t *seq_len;
+    const int64_t *cur_pos;
+    int32_t *status;
+} tri_kv_desc;
+
+/* Optional phase timing: events recorded on the call's stream before the
+ * first launch and after each phase of tri_compress_step.  Any member may be
+ * NULL.  The events must have been created by the caller. */
+typedef struct {
+    cudaEvent_t start;          /* before the query build                   */
+    cudaEvent_t after_query;    /* after the effective-query build          */
+    cudaEvent_t after_score;    /* after the score pass over all keys       */
+    cudaEvent_t after_evict;    /* after selection and compaction           */
+} tri_phase_events;
+
+/*
+ * tri_calibrate_centers - reduce pre-rotary query samples to head statistics
+ * ([Digest] "Core Mechanism", one-time centre calibration; "Key Concepts",
+ * Q/K Concentration; [GeoTrick] "The Core Idea", measured concentration).
+ *
+ *   q_pre : f32 [N][L][Hq][D] samples of the pre-rotary query (any N >= 1)
+ *   qbar  : f32 [L][Hq][D] out, the centre: mean sample (bands as dims i, i+64)
+ *   qabs  : f32 [L][Hq][D/2] out, A_i = mean over samples of |band i|
+ *   R     : f32 [L][Hq] out, concentration sum_i |qbar_i| / sum_i A_i in
+ *           [0, 1]; 1 when every sample is zero
+ * Accumulates in float64.  Works for keys too (pass key samples).
+ * Errors: TRI_ERR_INVALID (null pointer, N/L/Hq < 1, size overflow),
+ * TRI_ERR_UNSUPPORTED (D != 128), TRI_ERR_CUDA.
+ */
+tri_status tri_calibrate_centers(const float *q_pre, int N, int L, int Hq, int D,
+                                 float *qbar, float *qabs, float *R,
+                                 cudaStream_t stream);
+
+/*
+ * tri_build_query - the effective query of every unit, folded over its GQA
+ * group ([Digest] "Key Concepts", Trigonometric Distance Preference; future
+ * query positions p + delta averaged over the offset list):
+ *
+ *   m_i      = mean_delta exp(j theta_i (cur_pos[s] + delta))   (float64)
+ *   qeff     = real dims of mean_g qbar_{g,i} * m_i              [S][L][Hkv][D]
+ *   w_i      = mean_g (1 - R_g) (qabs_{g,i} - |qbar_{g,i}|)      [S][L][Hkv][D/2]
+ *
+ * so that the group score of a key K is qeff . K + sum_i w_i |K band i|.
+ *   qbar, qabs, R : statistics as produced by tri_calibrate_centers, for
+ *                   Hq = Hkv*G query heads
+ *   rope_base     : rotary base (> 0)
+ *   deltas        : HOST int32 [n_deltas], 1 <= n_deltas <= TRI_MAX_DELTAS;
+ *                   read during the call only
+ *   qeff, w       : f32 outputs, layouts above
+ * Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED, TRI_ERR_CUDA.
+ */
+tri_status tri_build_query(const tri_kv_desc *desc, const float *qbar, const float *qabs,
+                           const float *R, double rope_base, const int32_t *deltas,
+                           int n_deltas, float *qeff, float *w, cudaStream_t stream);
+
+/*
+ * tri_workspace_size - bytes of device workspace that tri_score and
+ * tri_compress_step need for this descriptor's shape.  The workspace must be
+ * 256-byte aligned.  Depends on S, L, Hkv and max_blocks only.
+ * Returns 0 for an invalid descriptor.
+ */
+size_t tri_workspace_size(const tri_kv_desc *desc, int budget);
+
+/*
+ * tri_score - score every cached key of every unit ([Digest] "Key
+ * Concepts"; [Abstract] "English"; [GeoTrick] "The Core Idea"):
+ *
+ *   s(t) = qeff . K_t + sum_i w_i sqrt(K_{t,i}^2 + K_{t,i+64}^2)
+ *
+ * which equals the mean over the G query heads of
+ *   sum_i Re(qbar_i m_i conj(K_t band i)) + (1 - R)(qabs_i - |qbar_i|)|K_t band i|.
+ * bf16 keys, fp32 arithmetic, streamed once from HBM.
+ *   scores : f32 [S][L][Hkv][max_blocks*16]; entry t of unit (s, l, h) is
+ *            written for t < seq_len[s]; the rest is left untouched.
+ *   workspace, ws_bytes : >= tri_workspace_size(desc, 1) bytes.
+ * Errors: as tri_build_query, plus TRI_ERR_WORKSPACE.  Device flags: BOUNDS
+ * (seq_len or a block id out of range: those keys are skipped), TIMEOUT.
+ */
+tri_status tri_score(const tri_kv_desc *desc, const float *qbar, const float *qabs,
+                     const float *R, double rope_base, const int32_t *deltas, int n_deltas,
+                     float *scores, void *workspace, size_t ws_bytes, cudaStream_t stream);
+
+/*
+ * tri_select_topk - the kept slots of every unit ([Digest] "Core Mechanism":
+ * keep only the top-scoring subset).  For a unit of len = seq_len[s] slots:
+ *   len <= budget : every slot is kept;
+ *   otherwise     : the last `window` slots, plus the (budget - window) best of
+ *                   the other slots by (score descending, slot ascending).
+ * -0 equals +0; a NaN score ranks as -infinity and sets TRI_DEVFLAG_NONFINITE.
+ *   scores : f32 [S][L][Hkv][max_blocks*16] (as written by tri_score)
+ *   budget : B >= 1, at most TRI_MAX_BUDGET; window: 0 <= W <= B
+ *   idx    : int32 [S][L][Hkv][budget] out; the kept slots ascending in the
+ *            first kept[s] entries, -1 after them
+ *   kept   : int32 [S] out; min(seq_len[s], budget)
+ * Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED, TRI_ERR_CUDA.
+ */
+tri_status tri_select_topk(const tri_kv_desc *desc, const float *scores, int budget,
+                           int window, int32_t *idx, int32_t *kept, cudaStream_t stream);
+
+/*
+ * tri_compact_kv - Forward-Packing Compaction ([GeoTrick] "Solving the
+ * Memory Fragmentation Problem"): for every unit and j < kept[s], row j of K
+ * and of V takes old row idx[j], in place across the sequence's blocks, in
+ * order.  Then seq_len[s] = kept[s], and the blocks
+ * block_table[s][ceil(kept/16) .. ceil(old_len/16)) are appended to
+ * freed_ids (sequence order, table order); *freed_count = their number.
+ *   idx   : int32 [S][L][Hkv][budget], each unit's first kept[s] entries
+ *           strictly ascending and < seq_len[s] (as from tri_select_topk)
+ *   kept  : int32 [S], 0 <= kept[s] <= seq_len[s]
+ *   freed_ids   : int32 [S*max_blocks] out;  freed_count : int32 [1] out
+ * The block table is not modified; the caller truncates it.
+ * Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED, TRI_ERR_CUDA.  Device flags:
+ * BOUNDS (an index, kept count or block id out of range: skipped).
+ */
+tri_status tri_compact_kv(tri_kv_desc *desc, const int32_t *idx, const int32_t *kept,
+                          int budget, int32_t *freed_ids, int32_t *freed_count,
+                          cudaStream_t stream);
+
+/*
+ * tri_compress_step - the whole step: effective query, score, select and
+ * compact for every unit of every sequence whose seq_len exceeds `budget`;
+ * shorter sequences are left untouched.  Same results as tri_score ->
+ * tri_select_topk -> tri_compact_kv, without materialising scores outside the
+ * workspace.
+ *   idx_out : optional int32 [S][L][Hkv][budget]; when not NULL receives the
+ *             kept slots of every compressed unit (entries of sequences left
+ *             untouched are not written)
+ *   events  : optional phase timing (see tri_phase_events)
+ *   workspace, ws_bytes : >= tri_workspace_size(desc, budget) bytes
+ * Errors and flags: union of the three calls above.
+ */
+tri_status tri_compress_step(tri_kv_desc *desc, const float *qbar, const float *qabs,
+                             const float *R, double rope_base, const int32_t *deltas,
+                             int n_deltas, int budget, int window, int32_t *freed_ids,
+                             int32_t *freed_count, int32_t *idx_out, void *workspace,
+                             size_t ws_bytes, const tri_phase_events *events,
+                             cudaStream_t stream);
+
+/*
+ * tri_sync_status - wait for `stream`, read the device status word, clear it,
+ * and return TRI_OK or the error its bits name (BOUNDS before TIMEOUT before
+ * NONFINITE).  TRI_ERR_CUDA if the stream itself reports an error.
+ */
+tri_status tri_sync_status(int32_t *status, cudaStream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char *tri_status_string(tri_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_ATTENTION_H */

@@ -1,0 +1,270 @@
+// score.cu - one streaming pass over every cached key.
+//
+// Pages: "TriAttention: Trigonometric KV Compression for Efficient Long
+// Reasoning" - "Key Concepts", Trigonometric Distance Preference and Norm as
+// Importance Signal; "TriAttention: Efficient Long Reasoning with
+// Trigonometric KV Compression" - "English" (centres score keys through a
+// trigonometric series, with Q/K norms as an additional signal);
+// "TriAttention: How a Geometric Trick Cuts LLM Memory Use by 10x Without
+// Losing Accuracy" - "The Core Idea" (norm signal weighted by measured
+// concentration).
+//
+// Score of a cached post-rotary key K (bf16, D = 128), from the folded
+// effective query of its unit (query.cu):
+//     s = sum_d qeff_d K_d + sum_i w_i sqrt(K_i^2 + K_{i+64}^2)
+//
+// Design (HBM-bound: 256 bytes and ~1.5 flop per byte):
+//  * Persistent CTAs, two per SM.  A work item is (sequence, layer, group of
+//    HG KV heads, run of 16 paged blocks); items are dealt round-robin.
+//  * Warp 8 is the producer: one lane issues one bulk copy (TMA engine, no
+//    multicast) per paged block, moving the HG contiguous 4 KiB (block, head)
+//    tiles of that block into a ring of shared-memory stages, with an
+//    evict-first L2 policy.  Full/empty mbarriers hand stages over.
+//  * Warps 0..7 consume: HG heads per stage, each warp owns one head (or a
+//    quarter of one), so its 24 coefficients stay in registers for the whole
+//    item.  8 lanes share a key: lane `sub` reads 16 bytes of the real half
+//    (dims 8sub..8sub+7) and the matching 16 bytes of the imaginary half
+//    (dims 64+8sub..), i.e. 8 whole bands; fp32 FMA; 3 xor-shuffles reduce.
+//  * Every wait is bounded; on a timeout the CTA records TRI_DEVFLAG_TIMEOUT,
+//    lets its in-flight copies land and returns.
+#include "tri_device.cuh"
+#include "tri_internal.h"
+
+namespace tri {
+
+namespace {
+
+constexpr int kConsumerWarps = 8;
+constexpr int kScoreThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStageBudgetBytes = 96 * 1024;
+constexpr int kMaxStages = 16;
+
+struct StageMeta {
+    int unit0;   // unit of the stage's first head
+    int t0;      // slot of the stage's first row
+    int nrows;   // valid rows (< 16 only in a sequence's last block)
+    int kind;    // 0: nothing to score, 1: keys, 2: end of work
+};
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1; it < kWaitLimitIters; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 0) {
+            if (*abort_flag) return false;
+            if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+        }
+    }
+    return false;
+}
+
+__device__ __forceinline__ float key_score(const uint4 a, const uint4 b, const float (&qr)[8],
+                                           const float (&qi)[8], const float (&ww)[8]) {
+    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
+    const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
+    float dot0 = 0.f, dot1 = 0.f, nrm0 = 0.f, nrm1 = 0.f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float r0 = bf16_lo(av[j]), r1 = bf16_hi(av[j]);
+        const float i0 = bf16_lo(bv[j]), i1 = bf16_hi(bv[j]);
+        dot0 = fmaf(qr[2 * j], r0, dot0);
+        dot1 = fmaf(qr[2 * j + 1], r1, dot1);
+        dot0 = fmaf(qi[2 * j], i0, dot0);
+        dot1 = fmaf(qi[2 * j + 1], i1, dot1);
+        nrm0 = fmaf(ww[2 * j], sqrt_fast(fmaf(r0, r0, i0 * i0)), nrm0);
+        nrm1 = fmaf(ww[2 * j + 1], sqrt_fast(fmaf(r1, r1, i1 * i1)), nrm1);
+    }
+    return (dot0 + dot1) + (nrm0 + nrm1);
+}
+
+__device__ void produce(const ScoreParams& p, uint8_t* tiles, uint64_t* full, uint64_t* empty, StageMeta* meta,
+                        volatile int* abort_flag) {
+    const int HG = p.heads_per_tile;
+    const uint32_t stages = (uint32_t)p.stages;
+    const uint32_t stage_bytes = (uint32_t)HG * kTileBytes;
+    const int n_hg = p.Hkv / HG;
+    const int total = p.item_off[p.S];
+    const uint64_t pol = l2_policy_evict_first();
+    uint32_t k = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
+        int lo = 0, hi = p.S;                    // item_off[lo] <= item < item_off[hi]
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.item_off[mid] <= item) lo = mid; else hi = mid;
+        }
+        const int s = lo;
+        const int len = p.len_ws[s];
+        const int nblk = (len + kBlockRows - 1) / kBlockRows;
+        const int nch = (nblk + kChunkBlocks - 1) / kChunkBlocks;
+        const int r = item - p.item_off[s];
+        const int chunk = r % nch, lhg = r / nch;
+        const int hg = lhg % n_hg, l = lhg / n_hg;
+        const int unit0 = (s * p.L + l) * p.Hkv + hg * HG;
+        const int b0 = chunk * kChunkBlocks;
+        const int b1 = min(b0 + kChunkBlocks, nblk);
+        for (int b = b0; b < b1; ++b) {
+            const uint32_t slot = k % stages;
+            if (k >= stages && !wait_or_abort(&empty[slot], ((k / stages) - 1) & 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (*abort_flag) {
+                ok = false;
+                break;
+            }
+            const int blk = p.block_table[(int64_t)s * p.max_blocks + b];
+            StageMeta m;
+            m.unit0 = unit0;
+            m.t0 = b * kBlockRows;
+            m.nrows = min(kBlockRows, len - b * kBlockRows);
+            if (blk >= 0 && blk < p.num_blocks) {
+                m.kind = 1;
+                meta[slot] = m;
+                mbar_arrive_expect_tx(&full[slot], stage_bytes);
+                const uint8_t* src =
+                    p.k_pool + ((((int64_t)l * p.num_blocks + blk) * p.Hkv + (int64_t)hg * HG) * kTileBytes);
+                bulk_copy_g2s(tiles + (size_t)slot * stage_bytes, src, stage_bytes, &full[slot], pol);
+            } else {
+                raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
+                m.kind = 0;
+                meta[slot] = m;
+                mbar_arrive(&full[slot]);
+            }
+            ++k;
+        }
+    }
+    if (ok) {
+        const uint32_t slot = k % stages;
+        if (k >= stages && !wait_or_abort(&empty[slot], ((k / stages) - 1) & 1u, abort_flag)) {
+            ok = false;
+        } else {
+            StageMeta m;
+            m.unit0 = 0;
+            m.t0 = 0;
+            m.nrows = 0;
+            m.kind = 2;
+            meta[slot] = m;
+            mbar_arrive(&full[slot]);
+        }
+    }
+    if (!ok) {
+        if (!*abort_flag) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
+        *abort_flag = 1;
+        // No copy may still be landing in this CTA's shared memory when it exits.
+        const uint32_t first = k > stages ? k - stages : 0u;
+        for (uint32_t j = first; j < k; ++j) mbar_wait_bounded(&full[j % stages], (j / stages) & 1u);
+    }
+}
+
+__device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t* tiles, uint64_t* full,
+                        uint64_t* empty, const StageMeta* meta, volatile int* abort_flag) {
+    const int HG = p.heads_per_tile;
+    const uint32_t stages = (uint32_t)p.stages;
+    const uint32_t stage_bytes = (uint32_t)HG * kTileBytes;
+    const int wph = kConsumerWarps / HG;       // warps per head
+    const int hig = warp / wph;                // head of the tile group
+    const int q0 = warp % wph;                 // first quad of keys
+    const int sub = lane & 7, kq = lane >> 3;
+    float qr[8], qi[8], ww[8];
+    int cur_unit = -1;
+    for (uint32_t k = 0;; ++k) {
+        const uint32_t slot = k % stages;
+        if (!wait_or_abort(&full[slot], (k / stages) & 1u, abort_flag)) {
+            if (!*abort_flag) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
+            *abort_flag = 1;
+            return;
+        }
+        const StageMeta m = meta[slot];
+        if (m.kind == 2) return;
+        if (m.kind == 1) {
+            const int unit = m.unit0 + hig;
+            if (unit != cur_unit) {
+                const float4* qe = reinterpret_cast<const float4*>(p.qeff + (int64_t)unit * kHeadDim);
+                const float4* we = reinterpret_cast<const float4*>(p.wts + (int64_t)unit * kBands);
+                const float4 x0 = qe[2 * sub], x1 = qe[2 * sub + 1];
+                const float4 y0 = qe[16 + 2 * sub], y1 = qe[16 + 2 * sub + 1];
+                const float4 z0 = we[2 * sub], z1 = we[2 * sub + 1];
+                qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
+                qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
+                qi[0] = y0.x; qi[1] = y0.y; qi[2] = y0.z; qi[3] = y0.w;
+                qi[4] = y1.x; qi[5] = y1.y; qi[6] = y1.z; qi[7] = y1.w;
+                ww[0] = z0.x; ww[1] = z0.y; ww[2] = z0.z; ww[3] = z0.w;
+                ww[4] = z1.x; ww[5] = z1.y; ww[6] = z1.z; ww[7] = z1.w;
+                cur_unit = unit;
+            }
+            const uint8_t* tile = tiles + (size_t)slot * stage_bytes + (size_t)hig * kTileBytes;
+            float* out = p.scores + (int64_t)unit * p.score_stride + m.t0;
+            for (int q = q0; q < 4; q += wph) {
+                const int row = q * 4 + kq;
+                const uint4 a = *reinterpret_cast<const uint4*>(tile + row * 256 + sub * 16);
+                const uint4 b = *reinterpret_cast<const uint4*>(tile + row * 256 + 128 + sub * 16);
+                float acc = key_score(a, b, qr, qi, ww);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+                acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+                if (sub == 0 && row < m.nrows) out[row] = acc;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+}
+
+__global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScoreParams p) {
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t stages = (uint32_t)p.stages;
+    const uint32_t stage_bytes = (uint32_t)p.heads_per_tile * kTileBytes;
+    uint8_t* tiles = smem;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + (size_t)stages * stage_bytes);
+    uint64_t* empty = full + stages;
+    StageMeta* meta = reinterpret_cast<StageMeta*>(empty + stages);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(meta + stages);
+    if (threadIdx.x == 0) {
+        for (uint32_t i = 0; i < stages; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], kConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (warp == kConsumerWarps) {
+        if (lane == 0) produce(p, tiles, full, empty, meta, abort_flag);
+        return;
+    }
+    consume(p, warp, lane, tiles, full, empty, meta, abort_flag);
+}
+
+size_t score_smem_bytes(int HG, int stages) {
+    return (size_t)stages * HG * kTileBytes + (size_t)stages * 2 * sizeof(uint64_t) +
+           (size_t)stages * sizeof(StageMeta) + 16;
+}
+
+}  // namespace
+
+int score_heads_per_tile(int Hkv) {
+    for (int hg = 8; hg > 1; hg >>= 1)
+        if (Hkv % hg == 0) return hg;
+    return 1;
+}
+
+cudaError_t launch_score(const ScoreParams& p_in, int max_items, int num_sms, cudaStream_t stream) {
+    ScoreParams p = p_in;
+    int stages = kStageBudgetBytes / (p.heads_per_tile * kTileBytes);
+    if (stages > kMaxStages) stages = kMaxStages;
+    if (stages < 2) stages = 2;
+    p.stages = stages;
+    const size_t smem = score_smem_bytes(p.heads_per_tile, stages);
+    cudaError_t e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int grid = num_sms * 2;
+    if (max_items < grid) grid = max_items;
+    if (grid < 1) grid = 1;
+    score_kernel<<<grid, kScoreThreads, smem, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace tri

@@ -1,0 +1,368 @@
+// tri_abi.cu - the extern "C" entry points declared in tri_attention.h.
+//
+// Host side only: argument checks (before any launch), workspace carving,
+// and the launch sequence of each call on the caller's stream.  Every
+// arithmetic step of the path runs in the kernels of calibrate.cu, query.cu,
+// score.cu and evict.cu.
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "tri_attention.h"
+#include "tri_internal.h"
+
+using namespace tri;
+
+namespace {
+
+constexpr size_t kWsAlign = 256;
+
+size_t align_up(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
+
+struct WsLayout {
+    size_t qeff, wts, len_ws, item_off, freed_off, scores, total;
+};
+
+WsLayout ws_layout(const tri_kv_desc* d) {
+    const size_t U = (size_t)d->S * d->L * d->Hkv;
+    const size_t max_len = (size_t)d->max_blocks * kBlockRows;
+    WsLayout w;
+    size_t off = 0;
+    w.qeff = off;      off = align_up(off + U * kHeadDim * sizeof(float));
+    w.wts = off;       off = align_up(off + U * kBands * sizeof(float));
+    w.len_ws = off;    off = align_up(off + (size_t)d->S * sizeof(int32_t));
+    w.item_off = off;  off = align_up(off + ((size_t)d->S + 1) * sizeof(int32_t));
+    w.freed_off = off; off = align_up(off + ((size_t)d->S + 1) * sizeof(int32_t));
+    w.scores = off;    off = align_up(off + U * max_len * sizeof(float));
+    w.total = off;
+    return w;
+}
+
+template <typename T>
+bool aligned(const T* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+tri_status check_desc(const tri_kv_desc* d) {
+    if (d == nullptr) return TRI_ERR_INVALID;
+    if (d->L < 1 || d->Hkv < 1 || d->G < 1 || d->S < 0 || d->num_blocks < 1 || d->max_blocks < 1)
+        return TRI_ERR_INVALID;
+    if (d->D != TRI_HEAD_DIM || d->block_size != TRI_BLOCK_SIZE) return TRI_ERR_UNSUPPORTED;
+    if (!d->k_pool || !d->v_pool || !d->block_table || !d->seq_len || !d->cur_pos || !d->status)
+        return TRI_ERR_INVALID;
+    if (!aligned(d->k_pool, 16) || !aligned(d->v_pool, 16) || !aligned(d->block_table, 4) ||
+        !aligned(d->seq_len, 4) || !aligned(d->cur_pos, 8) || !aligned(d->status, 4))
+        return TRI_ERR_INVALID;
+    const int64_t U = (int64_t)d->S * d->L * d->Hkv;
+    const int64_t Hq = (int64_t)d->Hkv * d->G;
+    const int64_t max_len = (int64_t)d->max_blocks * kBlockRows;
+    const int64_t items = (int64_t)d->S * d->L * d->Hkv * ((d->max_blocks + kChunkBlocks - 1) / kChunkBlocks);
+    if (U > INT_MAX || Hq > INT_MAX || max_len > INT_MAX || items > INT_MAX) return TRI_ERR_INVALID;
+    if ((int64_t)d->L * d->num_blocks * d->Hkv > INT64_MAX / kTileBytes) return TRI_ERR_INVALID;
+    return TRI_OK;
+}
+
+tri_status check_stats(const float* qbar, const float* qabs, const float* R) {
+    if (!qbar || !qabs || !R) return TRI_ERR_INVALID;
+    if (!aligned(qbar, 4) || !aligned(qabs, 4) || !aligned(R, 4)) return TRI_ERR_INVALID;
+    return TRI_OK;
+}
+
+tri_status check_query_args(double base, const int32_t* deltas, int n_deltas) {
+    if (!(base > 0.0) || !std::isfinite(base)) return TRI_ERR_INVALID;
+    if (deltas == nullptr || n_deltas < 1 || n_deltas > TRI_MAX_DELTAS) return TRI_ERR_INVALID;
+    return TRI_OK;
+}
+
+tri_status check_budget(int budget, int window) {
+    if (budget < 1 || window < 0 || window > budget) return TRI_ERR_INVALID;
+    if (budget > TRI_MAX_BUDGET) return TRI_ERR_UNSUPPORTED;
+    return TRI_OK;
+}
+
+tri_status check_workspace(const tri_kv_desc* d, const void* ws, size_t ws_bytes) {
+    if (ws == nullptr || ((uintptr_t)ws % kWsAlign) != 0) return TRI_ERR_WORKSPACE;
+    if (ws_bytes < ws_layout(d).total) return TRI_ERR_WORKSPACE;
+    return TRI_OK;
+}
+
+tri_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRI_OK : TRI_ERR_CUDA; }
+
+int device_sm_count() {
+    static std::mutex mu;
+    static int cache[128] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+QueryParams make_query_params(const tri_kv_desc* d, const float* qbar, const float* qabs, const float* R,
+                              double base, const int32_t* deltas, int n_deltas, float* qeff, float* wts) {
+    QueryParams q{};
+    q.qbar = qbar;
+    q.qabs = qabs;
+    q.R = R;
+    q.cur_pos = d->cur_pos;
+    q.base = base;
+    q.n_deltas = n_deltas;
+    for (int i = 0; i < n_deltas; ++i) q.deltas[i] = deltas[i];
+    q.qeff = qeff;
+    q.wts = wts;
+    q.L = d->L;
+    q.Hkv = d->Hkv;
+    q.G = d->G;
+    q.S = d->S;
+    q.seq_len = d->seq_len;
+    q.max_blocks = d->max_blocks;
+    q.heads_per_tile = score_heads_per_tile(d->Hkv);
+    q.status = d->status;
+    return q;
+}
+
+ScoreParams make_score_params(const tri_kv_desc* d, const uint8_t* ws, const WsLayout& w, float* scores,
+                              int64_t stride) {
+    ScoreParams s{};
+    s.k_pool = static_cast<const uint8_t*>(d->k_pool);
+    s.block_table = d->block_table;
+    s.len_ws = reinterpret_cast<const int32_t*>(ws + w.len_ws);
+    s.item_off = reinterpret_cast<const int32_t*>(ws + w.item_off);
+    s.qeff = reinterpret_cast<const float*>(ws + w.qeff);
+    s.wts = reinterpret_cast<const float*>(ws + w.wts);
+    s.scores = scores;
+    s.score_stride = stride;
+    s.status = d->status;
+    s.L = d->L;
+    s.Hkv = d->Hkv;
+    s.num_blocks = d->num_blocks;
+    s.S = d->S;
+    s.max_blocks = d->max_blocks;
+    s.heads_per_tile = score_heads_per_tile(d->Hkv);
+    return s;
+}
+
+int max_score_items(const tri_kv_desc* d) {
+    const int hg = score_heads_per_tile(d->Hkv);
+    const int64_t n = (int64_t)d->S * d->L * (d->Hkv / hg) * ((d->max_blocks + kChunkBlocks - 1) / kChunkBlocks);
+    return n > INT_MAX ? INT_MAX : (int)n;
+}
+
+EvictParams make_evict_params(const tri_kv_desc* d) {
+    EvictParams e{};
+    e.k_pool = static_cast<uint8_t*>(d->k_pool);
+    e.v_pool = static_cast<uint8_t*>(d->v_pool);
+    e.block_table = d->block_table;
+    e.L = d->L;
+    e.Hkv = d->Hkv;
+    e.num_blocks = d->num_blocks;
+    e.S = d->S;
+    e.max_blocks = d->max_blocks;
+    e.score_stride = (int64_t)d->max_blocks * kBlockRows;
+    e.status = d->status;
+    return e;
+}
+
+void record(cudaEvent_t ev, cudaStream_t stream) {
+    if (ev) cudaEventRecord(ev, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+tri_status tri_calibrate_centers(const float* q_pre, int N, int L, int Hq, int D, float* qbar, float* qabs,
+                                 float* R, cudaStream_t stream) {
+    if (!q_pre || N < 1 || L < 1 || Hq < 1) return TRI_ERR_INVALID;
+    if (D != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
+    if (check_stats(qbar, qabs, R) != TRI_OK || !aligned(q_pre, 4)) return TRI_ERR_INVALID;
+    if ((int64_t)L * Hq > INT_MAX) return TRI_ERR_INVALID;
+    return cuda_status(launch_calibrate(q_pre, N, L, Hq, qbar, qabs, R, stream));
+}
+
+tri_status tri_build_query(const tri_kv_desc* desc, const float* qbar, const float* qabs, const float* R,
+                           double rope_base, const int32_t* deltas, int n_deltas, float* qeff, float* w,
+                           cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if ((st = check_stats(qbar, qabs, R)) != TRI_OK) return st;
+    if ((st = check_query_args(rope_base, deltas, n_deltas)) != TRI_OK) return st;
+    if (!qeff || !w || !aligned(qeff, 16) || !aligned(w, 16)) return TRI_ERR_INVALID;
+    if (desc->S == 0) return TRI_OK;
+    QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas, qeff, w);
+    q.do_plan = 0;
+    return cuda_status(launch_query(q, stream));
+}
+
+size_t tri_workspace_size(const tri_kv_desc* desc, int budget) {
+    (void)budget;
+    if (check_desc(desc) != TRI_OK) return 0;
+    return ws_layout(desc).total;
+}
+
+tri_status tri_score(const tri_kv_desc* desc, const float* qbar, const float* qabs, const float* R,
+                     double rope_base, const int32_t* deltas, int n_deltas, float* scores, void* workspace,
+                     size_t ws_bytes, cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if ((st = check_stats(qbar, qabs, R)) != TRI_OK) return st;
+    if ((st = check_query_args(rope_base, deltas, n_deltas)) != TRI_OK) return st;
+    if (!scores || !aligned(scores, 4)) return TRI_ERR_INVALID;
+    if ((st = check_workspace(desc, workspace, ws_bytes)) != TRI_OK) return st;
+    if (desc->S == 0) return TRI_OK;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const WsLayout w = ws_layout(desc);
+    QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
+                                      reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
+    q.do_plan = 1;
+    q.budget = 0;
+    q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
+    q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
+    q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
+    q.freed_count = nullptr;
+    if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
+    ScoreParams sp = make_score_params(desc, ws, w, scores, (int64_t)desc->max_blocks * kBlockRows);
+    return cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream));
+}
+
+tri_status tri_select_topk(const tri_kv_desc* desc, const float* scores, int budget, int window, int32_t* idx,
+                           int32_t* kept, cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if ((st = check_budget(budget, window)) != TRI_OK) return st;
+    if (!scores || !idx || !kept || !aligned(scores, 4) || !aligned(idx, 4) || !aligned(kept, 4))
+        return TRI_ERR_INVALID;
+    if (desc->S == 0) return TRI_OK;
+    EvictParams e = make_evict_params(desc);
+    e.scores = scores;
+    e.lens = desc->seq_len;
+    e.budget = budget;
+    e.window = window;
+    e.idx_out = idx;
+    e.kept_out = kept;
+    e.do_select = 1;
+    e.do_compact = 0;
+    return cuda_status(launch_evict(e, stream));
+}
+
+tri_status tri_compact_kv(tri_kv_desc* desc, const int32_t* idx, const int32_t* kept, int budget,
+                          int32_t* freed_ids, int32_t* freed_count, cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if (budget < 1) return TRI_ERR_INVALID;
+    if (budget > TRI_MAX_BUDGET) return TRI_ERR_UNSUPPORTED;
+    if (!idx || !kept || !freed_ids || !freed_count || !aligned(idx, 4) || !aligned(kept, 4) ||
+        !aligned(freed_ids, 4) || !aligned(freed_count, 4))
+        return TRI_ERR_INVALID;
+    if (desc->S == 0) return cuda_status(cudaMemsetAsync(freed_count, 0, sizeof(int32_t), stream));
+    EvictParams e = make_evict_params(desc);
+    e.lens = desc->seq_len;
+    e.budget = budget;
+    e.idx_in = idx;
+    e.kept_in = kept;
+    e.do_select = 0;
+    e.do_compact = 1;
+    if ((st = cuda_status(launch_evict(e, stream))) != TRI_OK) return st;
+    FinalizeParams f{};
+    f.seq_len = desc->seq_len;
+    f.kept = kept;
+    f.block_table = desc->block_table;
+    f.S = desc->S;
+    f.max_blocks = desc->max_blocks;
+    f.freed_ids = freed_ids;
+    f.freed_count = freed_count;
+    f.status = desc->status;
+    return cuda_status(launch_finalize(f, stream));
+}
+
+tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* qabs, const float* R,
+                             double rope_base, const int32_t* deltas, int n_deltas, int budget, int window,
+                             int32_t* freed_ids, int32_t* freed_count, int32_t* idx_out, void* workspace,
+                             size_t ws_bytes, const tri_phase_events* events, cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if ((st = check_stats(qbar, qabs, R)) != TRI_OK) return st;
+    if ((st = check_query_args(rope_base, deltas, n_deltas)) != TRI_OK) return st;
+    if ((st = check_budget(budget, window)) != TRI_OK) return st;
+    if (!freed_ids || !freed_count || !aligned(freed_ids, 4) || !aligned(freed_count, 4)) return TRI_ERR_INVALID;
+    if (idx_out && !aligned(idx_out, 4)) return TRI_ERR_INVALID;
+    if ((st = check_workspace(desc, workspace, ws_bytes)) != TRI_OK) return st;
+    if (events) record(events->start, stream);
+    if (desc->S == 0) {
+        st = cuda_status(cudaMemsetAsync(freed_count, 0, sizeof(int32_t), stream));
+        if (events) {
+            record(events->after_query, stream);
+            record(events->after_score, stream);
+            record(events->after_evict, stream);
+        }
+        return st;
+    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const WsLayout w = ws_layout(desc);
+    QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
+                                      reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
+    q.do_plan = 1;
+    q.budget = budget;
+    q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
+    q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
+    q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
+    q.freed_count = freed_count;
+    if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
+    if (events) record(events->after_query, stream);
+
+    float* scores = reinterpret_cast<float*>(ws + w.scores);
+    ScoreParams sp = make_score_params(desc, ws, w, scores, (int64_t)desc->max_blocks * kBlockRows);
+    if ((st = cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream))) != TRI_OK)
+        return st;
+    if (events) record(events->after_score, stream);
+
+    EvictParams e = make_evict_params(desc);
+    e.scores = scores;
+    e.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
+    e.budget = budget;
+    e.window = window;
+    e.idx_out = idx_out;
+    e.do_select = 1;
+    e.do_compact = 1;
+    e.seq_len_out = desc->seq_len;
+    e.freed_off = reinterpret_cast<const int32_t*>(ws + w.freed_off);
+    e.freed_ids = freed_ids;
+    if ((st = cuda_status(launch_evict(e, stream))) != TRI_OK) return st;
+    if (events) record(events->after_evict, stream);
+    return TRI_OK;
+}
+
+tri_status tri_sync_status(int32_t* status, cudaStream_t stream) {
+    if (!status || !aligned(status, 4)) return TRI_ERR_INVALID;
+    int32_t h = 0;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return TRI_ERR_CUDA;
+    if (cudaMemcpyAsync(&h, status, sizeof(h), cudaMemcpyDeviceToHost, stream) != cudaSuccess) return TRI_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return TRI_ERR_CUDA;
+    if (h != 0) {
+        if (cudaMemsetAsync(status, 0, sizeof(int32_t), stream) != cudaSuccess) return TRI_ERR_CUDA;
+        if (cudaStreamSynchronize(stream) != cudaSuccess) return TRI_ERR_CUDA;
+    }
+    if (h & TRI_DEVFLAG_BOUNDS) return TRI_ERR_DEVICE_BOUNDS;
+    if (h & TRI_DEVFLAG_TIMEOUT) return TRI_ERR_TIMEOUT;
+    if (h & TRI_DEVFLAG_NONFINITE) return TRI_ERR_NONFINITE;
+    return TRI_OK;
+}
+
+const char* tri_status_string(tri_status s) {
+    switch (s) {
+        case TRI_OK: return "ok";
+        case TRI_ERR_INVALID: return "invalid argument";
+        case TRI_ERR_UNSUPPORTED: return "unsupported shape or size";
+        case TRI_ERR_CUDA: return "CUDA runtime error";
+        case TRI_ERR_DEVICE_BOUNDS: return "device saw an out-of-range index, length or block id";
+        case TRI_ERR_TIMEOUT: return "bounded device wait timed out";
+        case TRI_ERR_NONFINITE: return "NaN score";
+        case TRI_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

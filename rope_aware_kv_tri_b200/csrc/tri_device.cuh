@@ -1,0 +1,155 @@
+// tri_device.cuh - device-side building blocks shared by the kernels of the
+// TriAttention key-importance + eviction path (sm_100a only).
+//
+// Contents: mbarrier and bulk-copy (TMA engine, non-multicast) wrappers with
+// bounded waits, the device status word, bf16 unpacking, the order-preserving
+// key of an fp32 score, and block-wide integer scans.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tri_attention.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library is written for sm_100a (B200) only"
+#endif
+
+namespace tri {
+
+// Upper bound of every device wait on an mbarrier: a wait that has not
+// completed after this long records TRI_DEVFLAG_TIMEOUT and gives up.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;      // 2 s
+constexpr uint32_t kWaitLimitIters = 1u << 28;          // backstop
+
+__device__ __forceinline__ void raise_flag(int32_t* status, int flag) {
+    atomicOr(reinterpret_cast<int*>(status), flag);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_timer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// ---------------------------------------------------------------- mbarrier
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Wait for the phase of `bar` with the given parity to complete.  Returns
+// false (and waits no longer) after kWaitLimitNs or kWaitLimitIters.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1; it < kWaitLimitIters; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 31u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) return false;
+    }
+    return false;
+}
+
+// ------------------------------------------------------- bulk copy (TMA)
+// One contiguous global -> shared copy performed by the TMA engine; its
+// bytes are counted on `bar`.  Source and destination 16-byte aligned, size
+// a multiple of 16.  No cluster multicast.
+__device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                              uint64_t* bar, uint64_t l2_policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(smem_dst)),
+        "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(l2_policy)
+        : "memory");
+}
+
+// L2 policy for data read exactly once (the cached keys): evict first, so
+// that the small score scratch stays resident.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// ------------------------------------------------------------ arithmetic
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Square root through the MUFU unit (PTX sqrt.approx, subnormals flushed).
+__device__ __forceinline__ float sqrt_fast(float x) {
+    float r;
+    asm("sqrt.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Key of an fp32 score whose unsigned order is the score order: -0 is mapped
+// to +0 and NaN to -infinity, so equal scores get equal keys.
+__device__ __forceinline__ uint32_t order_key(float x) {
+    uint32_t b = __float_as_uint(x);
+    const uint32_t mag = b & 0x7fffffffu;
+    if (mag == 0u) b = 0u;
+    else if (mag > 0x7f800000u) b = 0xff800000u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+// Exclusive prefix sum over the block (NT threads, NT % 32 == 0).  `warp_tmp`
+// holds NT/32 ints of shared memory.  Returns this thread's exclusive prefix;
+// `total` receives the block total.  Contains two __syncthreads.
+template <int NT>
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_tmp, int& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_tmp[warp] = x;
+    __syncthreads();
+    int before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < NT / 32; ++w) {
+        const int c = warp_tmp[w];
+        before += (w < warp) ? c : 0;
+        tot += c;
+    }
+    __syncthreads();
+    total = tot;
+    return before + x - v;
+}
+
+}  // namespace tri

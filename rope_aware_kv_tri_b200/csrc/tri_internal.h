@@ -1,0 +1,101 @@
+// tri_internal.h - parameter blocks and launchers shared between the C ABI
+// (tri_abi.cu) and the kernel translation units.  Not installed; not ABI.
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tri_attention.h"
+
+namespace tri {
+
+constexpr int kHeadDim = TRI_HEAD_DIM;          // D
+constexpr int kBands = TRI_HEAD_DIM / 2;        // n
+constexpr int kBlockRows = TRI_BLOCK_SIZE;      // rows per paged block
+constexpr int kTileBytes = kBlockRows * kHeadDim * 2;   // one (block, head) tile: 4 KiB
+constexpr int kChunkBlocks = 16;                // paged blocks per score work item
+
+// --------------------------------------------------------------- queries
+struct QueryParams {
+    const float* qbar;        // [L][Hq][D]
+    const float* qabs;        // [L][Hq][D/2]
+    const float* R;           // [L][Hq]
+    const int64_t* cur_pos;   // [S]
+    double base;
+    int n_deltas;
+    int32_t deltas[TRI_MAX_DELTAS];
+    float* qeff;              // [U][D]
+    float* wts;               // [U][D/2]
+    int L, Hkv, G, S;
+    // plan (last block of the grid when do_plan != 0)
+    int do_plan;
+    const int32_t* seq_len;   // [S]
+    int max_blocks;
+    int budget;               // 0: plan every sequence (score only)
+    int heads_per_tile;       // HG
+    int32_t* len_ws;          // [S]
+    int32_t* item_off;        // [S+1]
+    int32_t* freed_off;       // [S+1]
+    int32_t* freed_count;     // [1] or null
+    int32_t* status;
+};
+cudaError_t launch_query(const QueryParams& p, cudaStream_t stream);
+
+// ----------------------------------------------------------------- score
+struct ScoreParams {
+    const uint8_t* k_pool;
+    const int32_t* block_table;
+    const int32_t* len_ws;
+    const int32_t* item_off;
+    const float* qeff;
+    const float* wts;
+    float* scores;
+    int64_t score_stride;     // floats between units in `scores`
+    int32_t* status;
+    int L, Hkv, num_blocks, S, max_blocks;
+    int heads_per_tile;       // HG, divides 8 and Hkv
+    int stages;
+};
+int score_heads_per_tile(int Hkv);
+cudaError_t launch_score(const ScoreParams& p, int max_items, int num_sms, cudaStream_t stream);
+
+// --------------------------------------------------- select + compaction
+struct EvictParams {
+    const float* scores;
+    int64_t score_stride;
+    const int32_t* lens;       // lengths the unit works from
+    int budget, window;
+    int32_t* idx_out;          // [U][budget] or null
+    int32_t* kept_out;         // [S] or null
+    const int32_t* idx_in;     // [U][budget] (compaction from given indices) or null
+    const int32_t* kept_in;    // [S] or null
+    int do_select, do_compact;
+    uint8_t* k_pool;
+    uint8_t* v_pool;
+    const int32_t* block_table;
+    int L, Hkv, num_blocks, S, max_blocks;
+    // step bookkeeping: CTA (s, 0, 0) writes seq_len[s] and the freed ids
+    int32_t* seq_len_out;      // or null
+    const int32_t* freed_off;  // [S+1] or null
+    int32_t* freed_ids;        // or null
+    int32_t* status;
+};
+cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream);
+
+// Freed-block list + new lengths after a standalone compaction.
+struct FinalizeParams {
+    int32_t* seq_len;
+    const int32_t* kept;
+    const int32_t* block_table;
+    int S, max_blocks;
+    int32_t* freed_ids;
+    int32_t* freed_count;
+    int32_t* status;
+};
+cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t stream);
+
+// ------------------------------------------------------------- calibrate
+cudaError_t launch_calibrate(const float* q, int N, int L, int Hq, float* qbar, float* qabs, float* R,
+                             cudaStream_t stream);
+
+}  // namespace tri

@@ -1,0 +1,137 @@
+"""The C-ABI library on the host (CPU only, no CUDA call is made).
+
+Checks that the in-tree shared library loads, exports every function that
+include/tri_attention.h declares, and rejects bad arguments on the host with
+the documented status before anything is launched.  The pointers passed are
+never dereferenced: every case here fails validation first.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import rope_aware_kv_tri_b200 as tri
+from rope_aware_kv_tri_b200 import build_lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "tri_attention.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_lib.build()
+    return tri.library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tri_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_function(lib):
+    names = declared_functions()
+    assert set(names) == set(tri.EXPORTS)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_status_strings(lib):
+    assert tri.tri_status_string(0) == "ok"
+    for code in range(1, 8):
+        assert tri.tri_status_string(code) not in ("ok", "unknown status")
+    assert tri.tri_status_string(99) == "unknown status"
+
+
+FAKE = 1 << 40           # 16-byte aligned, never dereferenced
+
+
+def _desc(**kw):
+    d = dict(L=2, Hkv=8, G=4, D=128, block_size=16, k_pool=FAKE, v_pool=FAKE + 4096, num_blocks=100,
+             block_table=FAKE, S=2, max_blocks=50, seq_len=FAKE, cur_pos=FAKE, status=FAKE)
+    d.update(kw)
+    return tri.TriKvDesc(**d)
+
+
+def _step(lib, desc, budget=64, window=8, deltas=(1, 2, 4), ws_bytes=None, base=1e4, stats=FAKE,
+          freed=FAKE, ws=FAKE):
+    arr = (ctypes.c_int32 * max(len(deltas), 1))(*deltas)
+    if ws_bytes is None:
+        ws_bytes = lib.tri_workspace_size(ctypes.byref(desc), budget) if desc is not None else 0
+    return lib.tri_compress_step(ctypes.byref(desc) if desc is not None else None, stats, FAKE, FAKE,
+                                 base, arr, len(deltas), budget, window, freed, FAKE, None, ws, ws_bytes,
+                                 None, None)
+
+
+def test_workspace_size(lib):
+    d = _desc()
+    n = lib.tri_workspace_size(ctypes.byref(d), 64)
+    U, max_len = 2 * 2 * 8, 50 * 16
+    assert n >= U * max_len * 4 + U * 192 * 4
+    assert n % 256 == 0
+    assert lib.tri_workspace_size(ctypes.byref(_desc(S=4)), 64) > n
+    assert lib.tri_workspace_size(ctypes.byref(_desc(D=64)), 64) == 0
+    assert lib.tri_workspace_size(None, 64) == 0
+
+
+@pytest.mark.parametrize("case,expect", [
+    (dict(desc=None), tri.TRI_ERR_INVALID),
+    (dict(D=64), tri.TRI_ERR_UNSUPPORTED),
+    (dict(block_size=32), tri.TRI_ERR_UNSUPPORTED),
+    (dict(L=0), tri.TRI_ERR_INVALID),
+    (dict(Hkv=0), tri.TRI_ERR_INVALID),
+    (dict(G=0), tri.TRI_ERR_INVALID),
+    (dict(S=-1), tri.TRI_ERR_INVALID),
+    (dict(num_blocks=0), tri.TRI_ERR_INVALID),
+    (dict(max_blocks=0), tri.TRI_ERR_INVALID),
+    (dict(k_pool=None), tri.TRI_ERR_INVALID),
+    (dict(v_pool=FAKE + 8), tri.TRI_ERR_INVALID),          # not 16-byte aligned
+    (dict(seq_len=None), tri.TRI_ERR_INVALID),
+    (dict(cur_pos=FAKE + 4), tri.TRI_ERR_INVALID),         # int64 misaligned
+    (dict(status=None), tri.TRI_ERR_INVALID),
+    (dict(max_blocks=1 << 28), tri.TRI_ERR_INVALID),       # slot count overflows int32
+    (dict(budget=0), tri.TRI_ERR_INVALID),
+    (dict(window=65), tri.TRI_ERR_INVALID),                 # window > budget
+    (dict(window=-1), tri.TRI_ERR_INVALID),
+    (dict(budget=20000, window=0), tri.TRI_ERR_UNSUPPORTED),
+    (dict(deltas=()), tri.TRI_ERR_INVALID),
+    (dict(deltas=tuple(range(1, 66))), tri.TRI_ERR_INVALID),
+    (dict(base=0.0), tri.TRI_ERR_INVALID),
+    (dict(base=float("nan")), tri.TRI_ERR_INVALID),
+    (dict(stats=None), tri.TRI_ERR_INVALID),
+    (dict(freed=None), tri.TRI_ERR_INVALID),
+    (dict(ws=None), tri.TRI_ERR_WORKSPACE),
+    (dict(ws=FAKE + 16), tri.TRI_ERR_WORKSPACE),           # not 256-byte aligned
+    (dict(ws_bytes=1024), tri.TRI_ERR_WORKSPACE),
+])
+def test_step_rejects_on_host(lib, case, expect):
+    case = dict(case)
+    desc_kw = {k: case.pop(k) for k in list(case) if k in tri.TriKvDesc.__dict__ or k in
+               ("L", "Hkv", "G", "D", "block_size", "k_pool", "v_pool", "num_blocks", "block_table", "S",
+                "max_blocks", "seq_len", "cur_pos", "status")}
+    desc = case.pop("desc") if "desc" in case else _desc(**desc_kw)
+    assert _step(lib, desc, **case) == expect
+
+
+def test_other_entry_points_reject_on_host(lib):
+    d = _desc()
+    dp = ctypes.byref(d)
+    arr = (ctypes.c_int32 * 1)(1)
+    assert lib.tri_calibrate_centers(None, 4, 1, 1, 128, FAKE, FAKE, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_calibrate_centers(FAKE, 0, 1, 1, 128, FAKE, FAKE, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_calibrate_centers(FAKE, 4, 1, 1, 96, FAKE, FAKE, FAKE, None) == tri.TRI_ERR_UNSUPPORTED
+    assert lib.tri_build_query(dp, FAKE, FAKE, FAKE, 1e4, arr, 1, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_score(dp, FAKE, FAKE, FAKE, 1e4, arr, 1, FAKE, FAKE, 16, None) == tri.TRI_ERR_WORKSPACE
+    assert lib.tri_select_topk(dp, FAKE, 8, 9, FAKE, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_select_topk(dp, None, 8, 2, FAKE, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_compact_kv(dp, FAKE, FAKE, 0, FAKE, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_compact_kv(dp, FAKE, FAKE, 8, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_sync_status(None, None) == tri.TRI_ERR_INVALID
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    import torch
+    with pytest.raises(ValueError):
+        tri.tri_calibrate_centers(torch.zeros(2, 1, 1, 128), torch.zeros(1, 1, 128), torch.zeros(1, 1, 64),
+                                  torch.zeros(1, 1))

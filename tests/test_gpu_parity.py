@@ -1,0 +1,320 @@
+"""GPU parity of every C-ABI entry point against the float64 oracle.
+
+All calls go through the shared library (rope_aware_kv_tri_b200 -> ctypes ->
+libtriattn.so).  Inputs are seeded synthetic workloads shaped like the five
+measured configurations, cut down so the oracle finishes in seconds while
+still spanning many 16-row blocks, several score work items, ragged tails,
+shuffled block tables, and every KV-heads-per-tile variant (8, 4, 2, 1).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_aware_kv_tri_b200 as tri
+from tests.gpu_helpers import (SCORE_TOL, cache_of, check_scores, check_selection, expected_pools_after,
+                               freed_expected, gpu_stats, oracle_stats, oracle_unit_scores, run_step,
+                               status_tensor, unit_rows)
+from workload import CONFIGS, make_workload
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+SMALL = {
+    "cfg1": CONFIGS["cfg1"],
+    "cfg2s": CONFIGS["cfg2"].replace(L=2, lens=[3001], budget=512, window=64, n_samples=512),
+    "cfg5s": CONFIGS["cfg5"].replace(L=2, lens=[700, 33, 1001, 16, 0, 530], budget=512, window=64,
+                                     n_samples=256, table="shuffled", pool_headroom=0.2),
+    "cfg4s": CONFIGS["cfg4"].replace(L=2, lens=[5000], budget=1024, window=256, n_samples=512),
+    "hkv6": CONFIGS["cfg2"].replace(L=2, Hkv=6, G=3, lens=[777, 1500], budget=300, window=20,
+                                    n_samples=256, table="shuffled"),
+    "hkv4": CONFIGS["cfg2"].replace(L=1, Hkv=4, G=2, lens=[1025], budget=100, window=0, n_samples=256),
+    "hkv3": CONFIGS["cfg2"].replace(L=1, Hkv=3, G=5, lens=[401, 17], budget=64, window=64, n_samples=128,
+                                    table="shuffled"),
+}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from rope_aware_kv_tri_b200 import build_lib
+    build_lib.build()
+    torch.cuda.init()
+
+
+def _workload(name, seed=0):
+    return make_workload(SMALL[name], device=DEV, seed=seed)
+
+
+# --------------------------------------------------------------- calibrate
+
+def test_calibrate_matches_oracle():
+    cfg = CONFIGS["cfg2"].replace(L=2, lens=[16], n_samples=777)
+    wl = make_workload(cfg, device=DEV)
+    qbar, qabs, R = gpu_stats(wl)
+    rb, ra, rr = oracle_stats(wl)
+    for got, ref in ((qbar, rb), (qabs, ra), (R, rr)):
+        got = got.double().cpu().numpy()
+        scale = np.abs(ref) + np.mean(np.abs(ref))
+        assert np.all(np.abs(got - ref) <= 1e-5 * scale)
+    assert np.all((rr > 0.3) & (rr <= 1.0))
+
+
+def test_calibrate_degenerate_samples():
+    q = torch.zeros(5, 1, 2, 128, device=DEV)
+    q[:, 0, 1] = torch.randn(128, device=DEV)       # head 1: identical samples
+    qbar = torch.empty(1, 2, 128, device=DEV)
+    qabs = torch.empty(1, 2, 64, device=DEV)
+    R = torch.empty(1, 2, device=DEV)
+    tri.tri_calibrate_centers(q, qbar, qabs, R)
+    torch.cuda.synchronize()
+    assert R[0, 0].item() == 1.0                    # all-zero samples
+    assert abs(R[0, 1].item() - 1.0) < 1e-6
+
+
+# ------------------------------------------------------------- build query
+
+@pytest.mark.parametrize("name", ["cfg1", "cfg5s", "hkv3"])
+def test_build_query_matches_oracle(name):
+    wl = _workload(name)
+    stats = gpu_stats(wl)
+    ref_stats = oracle_stats(wl)
+    S, L, Hkv, G = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv, wl.cfg.G
+    qeff = torch.empty(S, L, Hkv, 128, device=DEV)
+    w = torch.empty(S, L, Hkv, 64, device=DEV)
+    tri.tri_build_query(cache_of(wl), *stats, wl.cfg.base, wl.deltas, qeff, w)
+    qeff, w = qeff.double().cpu().numpy(), w.double().cpu().numpy()
+    qb, qa, rr = ref_stats
+    for s in range(S):
+        for l in range(L):
+            for h in range(Hkv):
+                sl = slice(h * G, (h + 1) * G)
+                rq, rw = oracle.group_query(qb[l, sl], qa[l, sl], rr[l, sl], int(wl.cur_pos[s]), wl.deltas,
+                                            wl.cfg.base)
+                sq = np.abs(rq).max() + 1e-30
+                sw = np.abs(rw).max() + 1e-30
+                assert np.abs(qeff[s, l, h] - rq).max() <= 2e-5 * sq
+                assert np.abs(w[s, l, h] - rw).max() <= 2e-5 * sw + 1e-7
+
+
+# ------------------------------------------------------------------ score
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_score_matches_oracle(name):
+    wl = _workload(name)
+    stats = gpu_stats(wl)
+    ref_stats = oracle_stats(wl)
+    cache = cache_of(wl)
+    S, L, Hkv = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv
+    max_len = wl.max_blocks * 16
+    sentinel = 12345.5
+    scores = torch.full((S, L, Hkv, max_len), sentinel, device=DEV)
+    ws = tri.alloc_workspace(cache, 1)
+    tri.tri_score(cache, *stats, wl.cfg.base, wl.deltas, scores, ws)
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    sc = scores.cpu().numpy()
+    table = wl.block_table.cpu().tolist()
+    worst = 0.0
+    for s in range(S):
+        n = int(wl.seq_len[s])
+        assert np.all(sc[s, :, :, n:] == sentinel), "score written past the sequence end"
+        for l in range(L):
+            for h in range(Hkv):
+                keys = unit_rows(wl.k_pool, table[s], n, l, h)
+                ref = oracle_unit_scores(wl, keys, ref_stats, s, l, h)
+                worst = max(worst, check_scores(sc[s, l, h, :n], ref))
+    print(f"{name}: worst score error / floor = {worst:.2e}")
+
+
+# ----------------------------------------------------------------- select
+
+def _score_fill(rng, n, kind):
+    if kind == "normal":
+        return rng.normal(size=n).astype(np.float32)
+    if kind == "ties":
+        return (np.round(rng.normal(size=n) * 4) / 4).astype(np.float32)
+    if kind == "zeros":
+        z = np.zeros(n, dtype=np.float32)
+        z[rng.random(n) < 0.5] = -0.0
+        return z
+    if kind == "wide":
+        return (rng.normal(size=n) * np.exp(rng.normal(size=n) * 20)).astype(np.float32)
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("budget,window", [(64, 8), (1, 0), (1, 1), (64, 64), (64, 0), (2048, 128)])
+def test_select_bit_exact_on_same_scores(budget, window):
+    rng = np.random.default_rng(budget * 131 + window)
+    lens = [0, 1, budget, budget + 1, 3 * budget + 5, 40000, 777, 5000]
+    kinds = ["normal", "ties", "zeros", "wide"]
+    S, L, Hkv = len(lens), 1, 4
+    max_blocks = -(-max(lens) // 16)
+    k = torch.zeros(1, 1, Hkv, 16, 128, dtype=torch.bfloat16, device=DEV)
+    table = torch.zeros(S, max_blocks, dtype=torch.int32, device=DEV)
+    seq_len = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    pos = torch.zeros(S, dtype=torch.int64, device=DEV)
+    cache = tri.KvCache(k, k.clone(), table, seq_len, pos, status_tensor(DEV), 1)
+    sc = np.full((S, L, Hkv, max_blocks * 16), np.nan, dtype=np.float32)
+    for s, n in enumerate(lens):
+        for h in range(Hkv):
+            sc[s, 0, h, :n] = _score_fill(rng, n, kinds[h])
+    scores = torch.from_numpy(sc).to(DEV)
+    idx = torch.full((S, L, Hkv, budget), -7, dtype=torch.int32, device=DEV)
+    kept = torch.full((S,), -7, dtype=torch.int32, device=DEV)
+    tri.tri_select_topk(cache, scores, budget, window, idx, kept)
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    idx, kept = idx.cpu().numpy(), kept.cpu().numpy()
+    for s, n in enumerate(lens):
+        assert kept[s] == min(n, budget)
+        for h in range(Hkv):
+            ref = oracle.select(sc[s, 0, h, :n].astype(np.float64), n, budget, window)
+            assert np.array_equal(idx[s, 0, h, :kept[s]], ref), (s, h, n)
+            assert np.all(idx[s, 0, h, kept[s]:] == -1)
+
+
+def test_select_nan_ranks_lowest_and_is_flagged():
+    n, budget, window = 300, 40, 5
+    rng = np.random.default_rng(3)
+    sc = rng.normal(size=(1, 1, 1, 304)).astype(np.float32)
+    sc[0, 0, 0, rng.choice(n - window, 280, replace=False)] = np.nan
+    k = torch.zeros(1, 1, 1, 16, 128, dtype=torch.bfloat16, device=DEV)
+    cache = tri.KvCache(k, k.clone(), torch.zeros(1, 19, dtype=torch.int32, device=DEV),
+                        torch.tensor([n], dtype=torch.int32, device=DEV), torch.zeros(1, dtype=torch.int64, device=DEV),
+                        status_tensor(DEV), 1)
+    idx = torch.empty(1, 1, 1, budget, dtype=torch.int32, device=DEV)
+    kept = torch.empty(1, dtype=torch.int32, device=DEV)
+    tri.tri_select_topk(cache, torch.from_numpy(sc).to(DEV), budget, window, idx, kept)
+    assert tri.tri_sync_status(cache.status) == tri.TRI_ERR_NONFINITE
+    ref = oracle.select(sc[0, 0, 0, :n].astype(np.float64), n, budget, window)
+    assert np.array_equal(idx[0, 0, 0].cpu().numpy(), ref)
+
+
+# ---------------------------------------------------------------- compact
+
+@pytest.mark.parametrize("name", ["cfg5s", "hkv6", "cfg1"])
+def test_compact_bit_exact_for_given_indices(name):
+    wl = _workload(name, seed=5)
+    budget, window = wl.cfg.budget, wl.cfg.window
+    S, L, Hkv = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv
+    lens = wl.seq_len.cpu().tolist()
+    rng = np.random.default_rng(9)
+    idx = np.full((S, L, Hkv, budget), -1, dtype=np.int32)
+    kept = [min(n, budget) for n in lens]
+    for s, n in enumerate(lens):
+        for l in range(L):
+            for h in range(Hkv):
+                if n <= budget:
+                    idx[s, l, h, :n] = np.arange(n)
+                else:
+                    pick = np.sort(rng.choice(n - window, budget - window, replace=False))
+                    if (s + l + h) % 3 == 0:       # a kept prefix that does not move
+                        pick = np.arange(budget - window)
+                    idx[s, l, h, :budget] = np.concatenate([pick, np.arange(n - window, n)])
+    pk, pv = wl.k_pool.clone(), wl.v_pool.clone()
+    cache = cache_of(wl)
+    freed = torch.full((S * wl.max_blocks,), -7, dtype=torch.int32, device=DEV)
+    count = torch.zeros(1, dtype=torch.int32, device=DEV)
+    idx_t = torch.from_numpy(idx).to(DEV)
+    tri.tri_compact_kv(cache, idx_t, torch.tensor(kept, dtype=torch.int32, device=DEV), budget, freed, count)
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    # the oracle moves the same rows on the bf16 bit patterns
+    kb, vb = pk.view(torch.int16).cpu().numpy(), pv.view(torch.int16).cpu().numpy()
+    nk, nv = kb.copy(), vb.copy()
+    table = wl.block_table.cpu().numpy()
+    for s, n in enumerate(lens):
+        for l in range(L):
+            for h in range(Hkv):
+                rows_k = oracle.unit_rows(kb, table[s], n, l, h)
+                rows_v = oracle.unit_rows(vb, table[s], n, l, h)
+                oracle.tri_oracle.store_unit_rows(nk, table[s], oracle.compact_rows(rows_k, idx[s, l, h, :kept[s]]), l, h)
+                oracle.tri_oracle.store_unit_rows(nv, table[s], oracle.compact_rows(rows_v, idx[s, l, h, :kept[s]]), l, h)
+    assert np.array_equal(wl.k_pool.view(torch.int16).cpu().numpy(), nk)
+    assert np.array_equal(wl.v_pool.view(torch.int16).cpu().numpy(), nv)
+    assert wl.seq_len.cpu().tolist() == kept
+    want = freed_expected(wl.block_table, lens, kept)
+    assert int(count.item()) == len(want) and freed[:len(want)].cpu().tolist() == want
+
+
+# ----------------------------------------------------------- compress step
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_compress_step_matches_oracle(name):
+    wl = _workload(name, seed=1)
+    budget, window = wl.cfg.budget, wl.cfg.window
+    stats = gpu_stats(wl)
+    ref_stats = oracle_stats(wl)
+    S, L, Hkv = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv
+    lens = wl.seq_len.cpu().tolist()
+    kept = [min(n, budget) for n in lens]
+    table = wl.block_table.cpu().tolist()
+    pk, pv = wl.k_pool.clone(), wl.v_pool.clone()
+    out = run_step(wl, stats, budget, window)
+    assert out["status"] == tri.TRI_OK
+    assert wl.seq_len.cpu().tolist() == kept
+    assert out["freed"] == freed_expected(wl.block_table, lens, kept)
+    idx = out["idx"]
+    differ = 0
+    for s, n in enumerate(lens):
+        for l in range(L):
+            for h in range(Hkv):
+                if n <= budget:
+                    assert torch.all(idx[s, l, h] == -7), "idx written for an untouched sequence"
+                    continue
+                ref = oracle_unit_scores(wl, unit_rows(pk, table[s], n, l, h), ref_stats, s, l, h)
+                differ += check_selection(idx[s, l, h].cpu().numpy(), ref, n, budget, window)
+    ek, ev = expected_pools_after(pk, pv, wl.block_table, lens, idx, kept)
+    assert torch.equal(wl.k_pool.view(torch.int16), ek.view(torch.int16))
+    assert torch.equal(wl.v_pool.view(torch.int16), ev.view(torch.int16))
+    print(f"{name}: {differ} kept slots differ from the oracle inside the cut band")
+
+
+def test_compress_step_all_equal_scores_keeps_earliest():
+    """Zero statistics make every score exactly 0: the step keeps the lowest
+    slots plus the window, exactly as the oracle."""
+    wl = _workload("cfg5s", seed=2)
+    L, Hq = wl.cfg.L, wl.cfg.Hq
+    zero = (torch.zeros(L, Hq, 128, device=DEV), torch.zeros(L, Hq, 64, device=DEV),
+            torch.ones(L, Hq, device=DEV))
+    lens = wl.seq_len.cpu().tolist()
+    out = run_step(wl, zero, 512, 64)
+    assert out["status"] == tri.TRI_OK
+    for s, n in enumerate(lens):
+        if n <= 512:
+            continue
+        want = np.concatenate([np.arange(448), np.arange(n - 64, n)])
+        for l in range(L):
+            for h in range(wl.cfg.Hkv):
+                assert np.array_equal(out["idx"][s, l, h].cpu().numpy(), want)
+
+
+def test_compress_step_budget_one_and_second_call_is_noop():
+    wl = _workload("cfg2s", seed=3)
+    stats = gpu_stats(wl)
+    out = run_step(wl, stats, 1, 1)
+    assert out["status"] == tri.TRI_OK and wl.seq_len.tolist() == [1]
+    k1 = wl.k_pool.clone()
+    out2 = run_step(wl, stats, 1, 1)
+    assert out2["freed"] == [] and torch.equal(k1, wl.k_pool)
+
+
+def test_bad_block_id_is_flagged_not_followed():
+    wl = _workload("cfg5s", seed=4)
+    stats = gpu_stats(wl)
+    wl.block_table[0, 3] = wl.num_blocks + 1000          # out of the pool
+    wl.block_table[2, 0] = -5
+    out = run_step(wl, stats, 512, 64)
+    assert out["status"] == tri.TRI_ERR_DEVICE_BOUNDS
+    # the context is intact: a clean call afterwards succeeds
+    wl2 = _workload("cfg2s", seed=4)
+    assert run_step(wl2, gpu_stats(wl2), 512, 64)["status"] == tri.TRI_OK
+
+
+def test_sequence_longer_than_its_table_is_flagged():
+    wl = _workload("cfg2s", seed=6)
+    stats = gpu_stats(wl)
+    wl.seq_len[0] = wl.max_blocks * 16 + 1
+    k0 = wl.k_pool.clone()
+    out = run_step(wl, stats, 512, 64)
+    assert out["status"] == tri.TRI_ERR_DEVICE_BOUNDS
+    assert torch.equal(k0, wl.k_pool)

@@ -1,0 +1,171 @@
+"""GPU parity on the decode loop and on the full-size workloads.
+
+* Decode loop: a CPU world (oracle) and a GPU world (C ABI) start from the
+  same seeded cache and receive the same appended tokens every round; each
+  world compresses with its own implementation, and the worlds are compared
+  after every round.  No oracle input ever comes from the GPU world.
+* Full size: the 32-layer x 8-head, T = 32768, B = 2048 workload in exactly
+  the launch configuration the benchmark times, plus the long-context and
+  wide-model workloads.  Every unit is checked for the properties that hold
+  at any size (lengths, freed blocks, window kept, rows moved bit-exactly
+  from their sources, nothing else touched); sampled units are checked
+  against the oracle score by score and index by index.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import rope_aware_kv_tri_b200 as tri
+from tests.gpu_helpers import (cache_of, check_scores, check_selection, expected_pools_after, freed_expected,
+                               gpu_stats, oracle_stats, oracle_unit_scores, run_step, unit_rows)
+from workload import CONFIGS, make_workload
+from workload.decode import append_tokens, recycle_freed
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from rope_aware_kv_tri_b200 import build_lib
+    build_lib.build()
+    torch.cuda.init()
+
+
+def test_decode_loop_two_worlds():
+    cfg = CONFIGS["cfg3"].replace(L=2, Hkv=4, G=2, lens=[0] * 4, lens_range=(300, 700), budget=256, window=32,
+                                  decode_append=64, decode_rounds=4, n_samples=256)
+    cpu = make_workload(cfg, device="cpu")
+    G, budget, window = cfg.G, cfg.budget, cfg.window
+    # GPU world: same starting state
+    gk, gv = cpu.k_pool.to(DEV), cpu.v_pool.to(DEV)
+    gtable, glen, gpos = cpu.block_table.to(DEV), cpu.seq_len.to(DEV), cpu.cur_pos.to(DEV)
+    samples = cpu.q_samples.to(DEV)
+    qbar = torch.empty(cfg.L, cfg.Hq, 128, device=DEV)
+    qabs = torch.empty(cfg.L, cfg.Hq, 64, device=DEV)
+    R = torch.empty(cfg.L, cfg.Hq, device=DEV)
+    tri.tri_calibrate_centers(samples, qbar, qabs, R)
+    rb, ra, rr = oracle.calibrate(cpu.q_samples.double().numpy())
+    S = cfg.S
+    for rnd in range(cfg.decode_rounds):
+        old = cpu.seq_len.tolist()
+        for s in range(S):
+            append_tokens(cpu, s, cfg.decode_append)
+        # mirror the appended rows, the table and the positions into the GPU world
+        gtable.copy_(cpu.block_table.to(DEV))
+        glen.copy_(cpu.seq_len.to(DEV))
+        gpos.copy_(cpu.cur_pos.to(DEV))
+        for s in range(S):
+            slots = torch.arange(old[s], old[s] + cfg.decode_append)
+            blk = cpu.block_table[s].long()[slots // 16]
+            row = slots % 16
+            gk[:, blk.to(DEV), :, row.to(DEV)] = cpu.k_pool[:, blk, :, row].to(DEV)
+            gv[:, blk.to(DEV), :, row.to(DEV)] = cpu.v_pool[:, blk, :, row].to(DEV)
+        lens = cpu.seq_len.tolist()
+        # GPU world step
+        cache = tri.KvCache(gk, gv, gtable, glen, gpos, torch.zeros(1, dtype=torch.int32, device=DEV), G)
+        ws = tri.alloc_workspace(cache, budget)
+        freed = torch.empty(S * cpu.max_blocks, dtype=torch.int32, device=DEV)
+        count = torch.empty(1, dtype=torch.int32, device=DEV)
+        idx = torch.empty(S, cfg.L, cfg.Hkv, budget, dtype=torch.int32, device=DEV)
+        tri.tri_compress_step(cache, qbar, qabs, R, cfg.base, cpu.deltas, budget, window, freed, count, ws,
+                              idx_out=idx)
+        assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+        # CPU world step (oracle)
+        res = oracle.compress_step(cpu.k_pool.double().numpy(), cpu.k_pool.view(torch.int16).numpy(),
+                                   cpu.v_pool.view(torch.int16).numpy(), cpu.block_table.numpy(), lens,
+                                   cpu.cur_pos.tolist(), rb, ra, rr, G, cpu.deltas, cfg.base, budget, window)
+        cpu.k_pool.view(torch.int16).copy_(torch.from_numpy(res["k_pool"]))
+        cpu.v_pool.view(torch.int16).copy_(torch.from_numpy(res["v_pool"]))
+        cpu.seq_len.copy_(torch.tensor(res["seq_len"], dtype=torch.int32))
+        n = int(count.item())
+        assert freed[:n].cpu().tolist() == res["freed_ids"]
+        assert glen.cpu().tolist() == res["seq_len"]
+        recycle_freed(cpu, lens, torch.tensor(res["freed_ids"] + [0], dtype=torch.int32), len(res["freed_ids"]))
+        differ = 0
+        for (s, l, h), ref_idx in res["idx"].items():
+            if lens[s] <= budget:
+                continue
+            differ += check_selection(idx[s, l, h].cpu().numpy(), res["scores"][(s, l, h)], lens[s], budget,
+                                      window)
+        if differ:
+            # an in-tolerance tie at a cut: the worlds now hold different rows
+            print(f"round {rnd}: worlds diverged inside the cut band ({differ} slots); stopping")
+            return
+        assert torch.equal(gk.view(torch.int16).cpu(), cpu.k_pool.view(torch.int16))
+        assert torch.equal(gv.view(torch.int16).cpu(), cpu.v_pool.view(torch.int16))
+        gtable.copy_(cpu.block_table.to(DEV))
+
+
+def _full_size(name, sample_units, check_all_rows):
+    cfg = CONFIGS[name]
+    wl = make_workload(cfg, device=DEV, seed=0)
+    stats = gpu_stats(wl)
+    budget, window = cfg.budget, cfg.window
+    S, L, Hkv, G = cfg.S, cfg.L, cfg.Hkv, cfg.G
+    lens = wl.seq_len.cpu().tolist()
+    kept = [min(n, budget) for n in lens]
+    table = wl.block_table.cpu().tolist()
+    rng = np.random.default_rng(0)
+    units = [(int(rng.integers(S)), int(rng.integers(L)), int(rng.integers(Hkv))) for _ in range(sample_units)]
+    units[0] = (0, 0, 0)
+    units[-1] = (S - 1, L - 1, Hkv - 1)
+    # pristine copies: of every row where affordable, else of the sampled units
+    if check_all_rows:
+        pk, pv = wl.k_pool.clone(), wl.v_pool.clone()
+    keys0 = {u: unit_rows(wl.k_pool, table[u[0]], lens[u[0]], u[1], u[2]).clone() for u in units}
+    vals0 = {u: unit_rows(wl.v_pool, table[u[0]], lens[u[0]], u[1], u[2]).clone() for u in units}
+    # scores of the sampled units from tri_score on the untouched cache
+    cache0 = cache_of(wl, seq_len=wl.seq_len.clone())
+    max_len = wl.max_blocks * 16
+    ws0 = tri.alloc_workspace(cache0, 1)
+    scores = torch.empty(S, L, Hkv, max_len, device=DEV)
+    tri.tri_score(cache0, *stats, cfg.base, wl.deltas, scores, ws0)
+    assert tri.tri_sync_status(cache0.status) == tri.TRI_OK
+    del ws0
+    out = run_step(wl, stats, budget, window)
+    assert out["status"] == tri.TRI_OK
+    assert wl.seq_len.cpu().tolist() == kept
+    assert out["freed"] == freed_expected(wl.block_table, lens, kept)
+    idx = out["idx"]
+    del out
+    if check_all_rows:
+        ek, ev = expected_pools_after(pk, pv, wl.block_table, lens, idx, kept)
+        del pk, pv
+        assert torch.equal(wl.k_pool.view(torch.int16), ek.view(torch.int16))
+        assert torch.equal(wl.v_pool.view(torch.int16), ev.view(torch.int16))
+        del ek, ev
+    # every unit: ascending, window kept
+    kept_idx = idx[..., :budget]
+    assert torch.all(kept_idx[..., 1:] > kept_idx[..., :-1])
+    cand = lens[0] - window
+    assert torch.all(kept_idx[..., budget - window:] == torch.arange(cand, lens[0], device=DEV, dtype=torch.int32))
+    for u in units:
+        s, l, h = u
+        n = lens[s]
+        ui = idx[s, l, h].long()
+        # moved rows are their sources, bit for bit
+        assert torch.equal(unit_rows(wl.k_pool, table[s], budget, l, h).view(torch.int16),
+                           keys0[u][ui].view(torch.int16))
+        assert torch.equal(unit_rows(wl.v_pool, table[s], budget, l, h).view(torch.int16),
+                           vals0[u][ui].view(torch.int16))
+        ref_stats = oracle_stats(wl, l, slice(h * G, (h + 1) * G))
+        ref = oracle.unit_scores(keys0[u].double().cpu().numpy(), *ref_stats, int(wl.cur_pos[s]), wl.deltas,
+                                 cfg.base)
+        err = check_scores(scores[s, l, h, :n].cpu().numpy(), ref)
+        differ = check_selection(ui.cpu().numpy(), ref, n, budget, window)
+        print(f"{name} unit {u}: worst score error/floor {err:.2e}, {differ} slots differ in the cut band")
+
+
+def test_full_size_32L_8H_T32768_B2048():
+    _full_size("cfg2", sample_units=8, check_all_rows=True)
+
+
+def test_full_size_long_context_T131072_B4096():
+    _full_size("cfg4", sample_units=4, check_all_rows=True)
+
+
+def test_full_size_wide_64L_G8_4x65536():
+    _full_size("cfg5", sample_units=4, check_all_rows=False)

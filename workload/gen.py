@@ -94,6 +94,34 @@ def noise_scale_for_target_concentration(centre_band_mag: np.ndarray, target: fl
     return 0.5 * (lo + hi)
 
 
+def _noise_scales(mags: np.ndarray, targets: np.ndarray) -> np.ndarray:
+    """``noise_scale_for_target_concentration`` for many heads at once."""
+    from scipy.special import i0e, i1e
+
+    def conc(sig):
+        a = mags * mags / (2.0 * sig[:, None] ** 2)
+        mean = sig[:, None] * math.sqrt(math.pi / 2.0) * ((1.0 + a) * i0e(a / 2.0) + a * i1e(a / 2.0))
+        return mags.sum(1) / mean.sum(1)
+
+    if np.any(targets <= 0.0) or np.any(targets > 1.0):
+        raise ValueError("target concentration must lie in (0, 1]")
+    lo = np.zeros(len(targets))
+    hi = np.ones(len(targets))
+    while True:
+        grow = conc(hi) > targets
+        if not grow.any():
+            break
+        hi[grow] *= 2.0
+    for _ in range(80):
+        mid = 0.5 * (lo + hi)
+        above = conc(np.maximum(mid, 1e-300)) > targets
+        lo = np.where(above, mid, lo)
+        hi = np.where(above, hi, mid)
+    out = 0.5 * (lo + hi)
+    out[targets >= 1.0] = 0.0
+    return out
+
+
 @dataclasses.dataclass
 class Workload:
     """Device tensors of one synthetic workload, laid out as the C ABI wants."""
@@ -186,10 +214,7 @@ def _query_statistics(cfg: WorkloadConfig, dev, gen: torch.Generator, rng: np.ra
         pick = rng.permutation(L * Hq)[:n_low]
         targets.reshape(-1)[pick] = cfg.low_r_value
     cmag = torch.sqrt(centres[..., :n] ** 2 + centres[..., n:] ** 2).cpu().numpy()
-    sigma = np.zeros((L, Hq))
-    for l in range(L):
-        for h in range(Hq):
-            sigma[l, h] = noise_scale_for_target_concentration(cmag[l, h], float(targets[l, h]))
+    sigma = _noise_scales(cmag.reshape(L * Hq, n), targets.reshape(-1)).reshape(L, Hq)
     sig = torch.tensor(sigma, dtype=torch.float64, device=dev)
     N = cfg.n_samples
     q = torch.empty(N, L, Hq, D, dtype=torch.float32, device=dev)
@@ -241,8 +266,11 @@ def make_workload(cfg: WorkloadConfig, device="cpu", seed: Optional[int] = None,
             table[s, :need[s]] = torch.tensor(blocks, dtype=torch.int32)
         free = [int(b) for b in perm[off:]]
 
-    k_pool = (torch.randn(L, NB, Hkv, bs, D, device=dev, generator=gen) * 2.0).to(torch.bfloat16)
-    v_pool = (torch.randn(L, NB, Hkv, bs, D, device=dev, generator=gen) * 2.0).to(torch.bfloat16)
+    k_pool = torch.empty(L, NB, Hkv, bs, D, dtype=torch.bfloat16, device=dev)
+    v_pool = torch.empty(L, NB, Hkv, bs, D, dtype=torch.bfloat16, device=dev)
+    for pool in (k_pool, v_pool):            # garbage in rows no token uses
+        for l in range(L):
+            pool[l].copy_(torch.randn(NB, Hkv, bs, D, device=dev, generator=gen) * 2.0)
     key_centres = torch.randn(L, Hkv, D, dtype=torch.float64, device=dev, generator=gen)
 
     q_samples, qbar, qabs, R = _query_statistics(cfg, dev, gen, rng, with_samples)
