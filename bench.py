@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the layer count (small profiling cases of the same kernels)")
     return ap.parse_args()
 
 
@@ -234,6 +236,8 @@ def run_ours(args, world, rank, local, dist):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     cfg = CONFIGS[args.workload]
+    if args.layers > 0:
+        cfg = cfg.replace(L=args.layers, name=f"{cfg.name} (L={args.layers})")
     if args.workload == "cfg3":
         raise SystemExit("the decode-loop workload is measured by tests/test_gpu_workloads.py, not here")
     wl = make_workload(cfg, device=dev, seed=rank)

@@ -26,7 +26,8 @@
  * Conventions shared by every entry point:
  *  - All array pointers are DEVICE memory owned by the caller, except where an
  *    argument says "host".  The library allocates no device memory: scratch
- *    comes from a caller-provided workspace sized by tri_workspace_size().
+ *    comes from a caller-provided workspace sized by tri_workspace_size()
+ *    (tri_compress_step_static_scratch uses a fixed array instead).
  *  - Every call is asynchronous on the cudaStream_t it is given (0 = the
  *    legacy default stream).  Host-side argument checks run before any
  *    launch; a rejected call launches nothing and changes nothing.
@@ -236,6 +237,40 @@ tri_status tri_compress_step(tri_kv_desc *desc, const float *qbar, const float *
                              int32_t *freed_count, int32_t *idx_out, void *workspace,
                              size_t ws_bytes, const tri_phase_events *events,
                              cudaStream_t stream);
+
+/*
+ * tri_compress_step_static_scratch - tri_compress_step without a workspace
+ * argument, for callers that cannot allocate device memory.  (The pages
+ * describe nothing like it: it exists only for how this library is called.)
+ *
+ * Who needs it: callers that have no way to obtain device scratch, such as
+ * a serving engine that hands nearly all HBM to its paged KV block pool at
+ * start-up and forbids allocation on the decode path, or a plain-C plugin
+ * loaded into such an engine without an allocator of its own.
+ *
+ * Instead of a caller workspace it uses one fixed array of
+ * TRI_STATIC_SCRATCH_BYTES of device memory built into the library; every
+ * GPU that loads the library holds that array until the process exits.
+ *   - Shapes whose tri_workspace_size(desc, budget) exceeds
+ *     TRI_STATIC_SCRATCH_BYTES are rejected with TRI_ERR_UNSUPPORTED before
+ *     anything is launched (use tri_compress_step with a workspace instead).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current and caches it; make
+ *     that first call before capturing the stream into a CUDA graph.
+ *   - All calls share the one array and it keeps the last call's contents.
+ *     Every call rewrites all of the scratch it reads, so nothing in it needs
+ *     to start at zero; but two calls whose work overlaps on the GPU (other
+ *     streams, other host threads) race on it and must not be issued.
+ *   - It allocates nothing: no cudaMalloc, cudaFree or allocating library
+ *     routine is called.
+ * Arguments, results, errors and device flags: as tri_compress_step (no
+ * phase events).
+ */
+#define TRI_STATIC_SCRATCH_BYTES (16u << 20)
+tri_status tri_compress_step_static_scratch(tri_kv_desc *desc, const float *qbar, const float *qabs,
+                                            const float *R, double rope_base, const int32_t *deltas,
+                                            int n_deltas, int budget, int window, int32_t *freed_ids,
+                                            int32_t *freed_count, int32_t *idx_out, cudaStream_t stream);
 
 /*
  * tri_sync_status - wait for `stream`, read the device status word, clear it,

@@ -37,9 +37,10 @@ TRI_MAX_BUDGET = 16384
 # Every symbol include/tri_attention.h declares.
 EXPORTS = (
     "tri_calibrate_centers", "tri_build_query", "tri_workspace_size", "tri_score",
-    "tri_select_topk", "tri_compact_kv", "tri_compress_step", "tri_sync_status",
-    "tri_status_string",
+    "tri_select_topk", "tri_compact_kv", "tri_compress_step", "tri_compress_step_static_scratch",
+    "tri_sync_status", "tri_status_string",
 )
+TRI_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class TriError(RuntimeError):
@@ -89,6 +90,7 @@ def _load() -> ctypes.CDLL:
         "tri_compact_kv": (I, [desc_p, P, P, I, P, P, P]),
         "tri_compress_step": (I, [desc_p, P, P, P, D, P, I, I, I, P, P, P, P, S,
                                   ctypes.POINTER(TriPhaseEvents), P]),
+        "tri_compress_step_static_scratch": (I, [desc_p, P, P, P, D, P, I, I, I, P, P, P, P]),
         "tri_sync_status": (I, [P, P]),
         "tri_status_string": (ctypes.c_char_p, [I]),
     }
@@ -244,6 +246,21 @@ def tri_compress_step(cache: KvCache, qbar, qabs, R, rope_base: float, deltas, b
         _ptr(idx_out, torch.int32, "idx_out", allow_none=True),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), ev, _stream(stream))
     _check(code, "tri_compress_step")
+
+
+def tri_compress_step_static_scratch(cache: KvCache, qbar, qabs, R, rope_base: float, deltas, budget: int,
+                                     window: int, freed_ids, freed_count, idx_out=None, stream=None) -> None:
+    """tri_compress_step without a workspace argument: the library's own
+    fixed device scratch (TRI_STATIC_SCRATCH_BYTES) is used instead, for
+    callers that cannot allocate device memory.  Calls must not overlap on
+    the GPU; the first call on a device should precede any graph capture."""
+    arr, n = _deltas(deltas)
+    code = library().tri_compress_step_static_scratch(
+        cache.ref, _ptr(qbar, torch.float32, "qbar"), _ptr(qabs, torch.float32, "qabs"),
+        _ptr(R, torch.float32, "R"), float(rope_base), arr, n, int(budget), int(window),
+        _ptr(freed_ids, torch.int32, "freed_ids"), _ptr(freed_count, torch.int32, "freed_count"),
+        _ptr(idx_out, torch.int32, "idx_out", allow_none=True), _stream(stream))
+    _check(code, "tri_compress_step_static_scratch")
 
 
 def tri_sync_status(status, stream=None) -> int:
