@@ -374,7 +374,7 @@ def run_ours(args, world, rank, local, dist):
                    "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
                    "timing": "CUDA events around each tri_compress_step; kept-region restore untimed"},
         "roofline": roofline, "step_roofline": step_roofline,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clk,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 5 * args.steps, "clocks": clk,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)

@@ -189,7 +189,8 @@ tri_status tri_score(const tri_kv_desc *desc, const float *qbar, const float *qa
  *   otherwise     : the last `window` slots, plus the (budget - window) best of
  *                   the other slots by (score descending, slot ascending).
  * -0 equals +0; a NaN score ranks as -infinity and sets TRI_DEVFLAG_NONFINITE.
- *   scores : f32 [S][L][Hkv][max_blocks*16] (as written by tri_score)
+ *   scores : f32 [S][L][Hkv][max_blocks*16] (as written by tri_score),
+ *            16-byte aligned
  *   budget : B >= 1, at most TRI_MAX_BUDGET; window: 0 <= W <= B
  *   idx    : int32 [S][L][Hkv][budget] out; the kept slots ascending in the
  *            first kept[s] entries, -1 after them

@@ -8,7 +8,7 @@
 // Losing Accuracy" - "The Core Idea" (norm signal weighted by the measured
 // concentration).
 //
-// For unit (s, l, h) and band i (one thread each):
+// For unit (s, l, h) and band i:
 //   m_i  = mean_delta exp(j theta_i (p_s + delta)),  theta_i = base^(-2i/D)
 //   qeff = real dims of mean_g qbar_{g,i} m_i          (bands i -> dims i, i+64)
 //   w_i  = mean_g (1 - R_g)(qabs_{g,i} - |qbar_{g,i}|)
@@ -30,22 +30,36 @@ namespace {
 constexpr int kQueryThreads = 256;
 constexpr int kUnitsPerCta = kQueryThreads / kBands;   // 4
 
-__device__ void build_unit_query(const QueryParams& p, int u) {
+// CTA b builds units [4k, 4k + 4) of sequence s (k = b mod ctas_per_seq):
+// the phase mean m_i of the sequence is shared, its offsets split over the
+// four 64-thread groups; then group g folds unit 4k + g.
+__device__ void build_unit_queries(const QueryParams& p, int b, int ctas_per_seq) {
+    __shared__ double s_mr[kUnitsPerCta][kBands], s_mi[kUnitsPerCta][kBands];
     const int i = threadIdx.x % kBands;
+    const int grp = threadIdx.x / kBands;
     const int LH = p.L * p.Hkv;
-    const int s = u / LH, rem = u % LH, l = rem / p.Hkv, h = rem % p.Hkv;
-    const int Hq = p.Hkv * p.G;
+    const int s = b / ctas_per_seq;
     const int64_t pos = p.cur_pos[s];
     const double theta = pow(p.base, -2.0 * (double)i / (double)kHeadDim);
     double mr = 0.0, mi = 0.0;
-    for (int d = 0; d < p.n_deltas; ++d) {
+    for (int d = grp; d < p.n_deltas; d += kUnitsPerCta) {
         double sn, cs;
         sincos(theta * (double)(pos + (int64_t)p.deltas[d]), &sn, &cs);
         mr += cs;
         mi += sn;
     }
+    s_mr[grp][i] = mr;
+    s_mi[grp][i] = mi;
+    __syncthreads();
+    mr = (s_mr[0][i] + s_mr[1][i]) + (s_mr[2][i] + s_mr[3][i]);
+    mi = (s_mi[0][i] + s_mi[1][i]) + (s_mi[2][i] + s_mi[3][i]);
     mr /= p.n_deltas;
     mi /= p.n_deltas;
+    const int k = (b % ctas_per_seq) * kUnitsPerCta + grp;     // unit within the sequence
+    if (k >= LH) return;
+    const int u = s * LH + k;
+    const int l = k / p.Hkv, h = k % p.Hkv;
+    const int Hq = p.Hkv * p.G;
     double cr = 0.0, ci = 0.0, wa = 0.0;
     for (int g = 0; g < p.G; ++g) {
         const int64_t row = (int64_t)l * Hq + (int64_t)h * p.G + g;
@@ -59,6 +73,10 @@ __device__ void build_unit_query(const QueryParams& p, int u) {
     p.qeff[(int64_t)u * kHeadDim + i] = (float)(cr * invG);
     p.qeff[(int64_t)u * kHeadDim + i + kBands] = (float)(ci * invG);
     p.wts[(int64_t)u * kBands + i] = (float)(wa * invG);
+    if (i == 0 && p.unit_kmin) {
+        p.unit_kmin[u] = 0xffffffffu;
+        p.unit_kmax[u] = 0u;
+    }
 }
 
 __device__ void plan_sequences(const QueryParams& p) {
@@ -99,25 +117,27 @@ __device__ void plan_sequences(const QueryParams& p) {
         p.item_off[p.S] = carry_items;
         p.freed_off[p.S] = carry_freed;
         if (p.freed_count) *p.freed_count = carry_freed;
+        if (p.zero_words) {
+            p.zero_words[0] = 0;
+            p.zero_words[1] = 0;
+        }
     }
 }
 
-__global__ void __launch_bounds__(kQueryThreads) query_kernel(const QueryParams p, int n_query_ctas) {
+__global__ void __launch_bounds__(kQueryThreads) query_kernel(const QueryParams p, int ctas_per_seq) {
+    const int n_query_ctas = p.S * ctas_per_seq;
     if ((int)blockIdx.x == n_query_ctas) {
         plan_sequences(p);
         return;
     }
-    const int U = p.S * p.L * p.Hkv;
-    const int u = blockIdx.x * kUnitsPerCta + threadIdx.x / kBands;
-    if (u < U) build_unit_query(p, u);
+    build_unit_queries(p, blockIdx.x, ctas_per_seq);
 }
 
 }  // namespace
 
 cudaError_t launch_query(const QueryParams& p, cudaStream_t stream) {
-    const int U = p.S * p.L * p.Hkv;
-    const int nq = (U + kUnitsPerCta - 1) / kUnitsPerCta;
-    query_kernel<<<nq + (p.do_plan ? 1 : 0), kQueryThreads, 0, stream>>>(p, nq);
+    const int per_seq = (p.L * p.Hkv + kUnitsPerCta - 1) / kUnitsPerCta;
+    query_kernel<<<p.S * per_seq + (p.do_plan ? 1 : 0), kQueryThreads, 0, stream>>>(p, per_seq);
     return cudaGetLastError();
 }
 

@@ -19,12 +19,17 @@
 //  * Warp 8 is the producer: one lane issues one bulk copy (TMA engine, no
 //    multicast) per paged block, moving the HG contiguous 4 KiB (block, head)
 //    tiles of that block into a ring of shared-memory stages, with an
-//    evict-first L2 policy.  Full/empty mbarriers hand stages over.
+//    evict-first L2 policy (scores are stored evict-last, so the selection
+//    finds them in L2).  Full/empty mbarriers hand stages over.
 //  * Warps 0..7 consume: HG heads per stage, each warp owns one head (or a
 //    quarter of one), so its 24 coefficients stay in registers for the whole
 //    item.  8 lanes share a key: lane `sub` reads 16 bytes of the real half
 //    (dims 8sub..8sub+7) and the matching 16 bytes of the imaginary half
 //    (dims 64+8sub..), i.e. 8 whole bands; fp32 FMA; 3 xor-shuffles reduce.
+//  * Each warp also tracks the smallest and largest order key of the scores
+//    it writes for a unit and folds them into the unit's key range with one
+//    atomicMin/atomicMax per item; the selection buckets scores linearly over
+//    that range.
 //  * Every wait is bounded; on a timeout the CTA records TRI_DEVFLAG_TIMEOUT,
 //    lets its in-flight copies land and returns.
 #include "tri_device.cuh"
@@ -169,6 +174,19 @@ __device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t*
     const int sub = lane & 7, kq = lane >> 3;
     float qr[8], qi[8], ww[8];
     int cur_unit = -1;
+    const uint64_t keep_pol = l2_policy_evict_last();   // scores are re-read by the selection
+    // order-key range of the scores this warp wrote for cur_unit
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    auto flush_range = [&]() {
+        const uint32_t lo = __reduce_min_sync(0xffffffffu, kmin);
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0 && cur_unit >= 0 && lo <= hi) {
+            atomicMin(&p.unit_kmin[cur_unit], lo);
+            atomicMax(&p.unit_kmax[cur_unit], hi);
+        }
+        kmin = 0xffffffffu;
+        kmax = 0u;
+    };
     for (uint32_t k = 0;; ++k) {
         const uint32_t slot = k % stages;
         if (!wait_or_abort(&full[slot], (k / stages) & 1u, abort_flag)) {
@@ -177,10 +195,14 @@ __device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t*
             return;
         }
         const StageMeta m = meta[slot];
-        if (m.kind == 2) return;
+        if (m.kind == 2) {
+            flush_range();
+            return;
+        }
         if (m.kind == 1) {
             const int unit = m.unit0 + hig;
             if (unit != cur_unit) {
+                flush_range();
                 const float4* qe = reinterpret_cast<const float4*>(p.qeff + (int64_t)unit * kHeadDim);
                 const float4* we = reinterpret_cast<const float4*>(p.wts + (int64_t)unit * kBands);
                 const float4 x0 = qe[2 * sub], x1 = qe[2 * sub + 1];
@@ -204,7 +226,12 @@ __device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t*
                 acc += __shfl_xor_sync(0xffffffffu, acc, 1);
                 acc += __shfl_xor_sync(0xffffffffu, acc, 2);
                 acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-                if (sub == 0 && row < m.nrows) out[row] = acc;
+                if (sub == 0 && row < m.nrows) {
+                    store_with_policy(out + row, acc, keep_pol);
+                    const uint32_t key = order_key(acc);
+                    kmin = min(kmin, key);
+                    kmax = max(kmax, key);
+                }
             }
         }
         __syncwarp();

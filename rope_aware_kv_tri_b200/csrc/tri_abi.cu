@@ -21,10 +21,20 @@ constexpr size_t kWsAlign = 256;
 size_t align_up(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
 
 struct WsLayout {
-    size_t qeff, wts, len_ws, item_off, freed_off, scores, total;
+    size_t qeff, wts, len_ws, item_off, freed_off, kmin, kmax, scores, idx, words, info, owner, scratch, total;
+    int scratch_rows;
 };
 
-WsLayout ws_layout(const tri_kv_desc* d) {
+// Rows of the compaction scratch: a quarter of the kept rows of all units
+// (units that do not fit compact their at-risk prefix in place instead).
+int scratch_rows_for(const tri_kv_desc* d, int budget) {
+    const int64_t rows = (int64_t)d->S * d->L * d->Hkv * (budget > 0 ? budget : 0) / 4;
+    if (budget <= 0) return 0;
+    return (int)(rows < 64 ? 64 : (rows > (1 << 24) ? (1 << 24) : rows));
+}
+
+// Workspace of a step with budget `budget` (0: the score-only part).
+WsLayout ws_layout(const tri_kv_desc* d, int budget) {
     const size_t U = (size_t)d->S * d->L * d->Hkv;
     const size_t max_len = (size_t)d->max_blocks * kBlockRows;
     WsLayout w;
@@ -34,7 +44,16 @@ WsLayout ws_layout(const tri_kv_desc* d) {
     w.len_ws = off;    off = align_up(off + (size_t)d->S * sizeof(int32_t));
     w.item_off = off;  off = align_up(off + ((size_t)d->S + 1) * sizeof(int32_t));
     w.freed_off = off; off = align_up(off + ((size_t)d->S + 1) * sizeof(int32_t));
+    w.kmin = off;      off = align_up(off + U * sizeof(uint32_t));
+    w.kmax = off;      off = align_up(off + U * sizeof(uint32_t));
     w.scores = off;    off = align_up(off + U * max_len * sizeof(float));
+    w.idx = off;       off = align_up(off + U * (size_t)(budget > 0 ? budget : 0) * sizeof(int32_t));
+    w.scratch_rows = scratch_rows_for(d, budget);
+    const size_t per_unit = budget > 0 ? 1 : 0;
+    w.words = off;     off = align_up(off + 2 * sizeof(int32_t) * per_unit);
+    w.info = off;      off = align_up(off + U * 4 * sizeof(int32_t) * per_unit);
+    w.owner = off;     off = align_up(off + (size_t)w.scratch_rows * 2 * sizeof(int32_t));
+    w.scratch = off;   off = align_up(off + (size_t)w.scratch_rows * 2 * kHeadDim * 2);
     w.total = off;
     return w;
 }
@@ -79,9 +98,9 @@ tri_status check_budget(int budget, int window) {
     return TRI_OK;
 }
 
-tri_status check_workspace(const tri_kv_desc* d, const void* ws, size_t ws_bytes) {
+tri_status check_workspace(const tri_kv_desc* d, const void* ws, size_t ws_bytes, int budget) {
     if (ws == nullptr || ((uintptr_t)ws % kWsAlign) != 0) return TRI_ERR_WORKSPACE;
-    if (ws_bytes < ws_layout(d).total) return TRI_ERR_WORKSPACE;
+    if (ws_bytes < ws_layout(d, budget).total) return TRI_ERR_WORKSPACE;
     return TRI_OK;
 }
 
@@ -135,6 +154,8 @@ ScoreParams make_score_params(const tri_kv_desc* d, const uint8_t* ws, const WsL
     s.wts = reinterpret_cast<const float*>(ws + w.wts);
     s.scores = scores;
     s.score_stride = stride;
+    s.unit_kmin = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(ws) + w.kmin);
+    s.unit_kmax = reinterpret_cast<uint32_t*>(const_cast<uint8_t*>(ws) + w.kmax);
     s.status = d->status;
     s.L = d->L;
     s.Hkv = d->Hkv;
@@ -164,6 +185,22 @@ EvictParams make_evict_params(const tri_kv_desc* d) {
     e.score_stride = (int64_t)d->max_blocks * kBlockRows;
     e.status = d->status;
     return e;
+}
+
+MoveParams make_move_params(const tri_kv_desc* d, const int32_t* idx, int budget) {
+    MoveParams m{};
+    m.idx = idx;
+    m.budget = budget;
+    m.k_pool = static_cast<uint8_t*>(d->k_pool);
+    m.v_pool = static_cast<uint8_t*>(d->v_pool);
+    m.block_table = d->block_table;
+    m.L = d->L;
+    m.Hkv = d->Hkv;
+    m.num_blocks = d->num_blocks;
+    m.S = d->S;
+    m.max_blocks = d->max_blocks;
+    m.status = d->status;
+    return m;
 }
 
 void record(cudaEvent_t ev, cudaStream_t stream) {
@@ -198,9 +235,8 @@ tri_status tri_build_query(const tri_kv_desc* desc, const float* qbar, const flo
 }
 
 size_t tri_workspace_size(const tri_kv_desc* desc, int budget) {
-    (void)budget;
-    if (check_desc(desc) != TRI_OK) return 0;
-    return ws_layout(desc).total;
+    if (check_desc(desc) != TRI_OK || budget < 0 || budget > TRI_MAX_BUDGET) return 0;
+    return ws_layout(desc, budget).total;
 }
 
 tri_status tri_score(const tri_kv_desc* desc, const float* qbar, const float* qabs, const float* R,
@@ -211,10 +247,10 @@ tri_status tri_score(const tri_kv_desc* desc, const float* qbar, const float* qa
     if ((st = check_stats(qbar, qabs, R)) != TRI_OK) return st;
     if ((st = check_query_args(rope_base, deltas, n_deltas)) != TRI_OK) return st;
     if (!scores || !aligned(scores, 4)) return TRI_ERR_INVALID;
-    if ((st = check_workspace(desc, workspace, ws_bytes)) != TRI_OK) return st;
+    if ((st = check_workspace(desc, workspace, ws_bytes, 0)) != TRI_OK) return st;
     if (desc->S == 0) return TRI_OK;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const WsLayout w = ws_layout(desc);
+    const WsLayout w = ws_layout(desc, 0);
     QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
                                       reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
     q.do_plan = 1;
@@ -223,6 +259,8 @@ tri_status tri_score(const tri_kv_desc* desc, const float* qbar, const float* qa
     q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
     q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
     q.freed_count = nullptr;
+    q.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
+    q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     ScoreParams sp = make_score_params(desc, ws, w, scores, (int64_t)desc->max_blocks * kBlockRows);
     return cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream));
@@ -233,7 +271,7 @@ tri_status tri_select_topk(const tri_kv_desc* desc, const float* scores, int bud
     tri_status st = check_desc(desc);
     if (st != TRI_OK) return st;
     if ((st = check_budget(budget, window)) != TRI_OK) return st;
-    if (!scores || !idx || !kept || !aligned(scores, 4) || !aligned(idx, 4) || !aligned(kept, 4))
+    if (!scores || !idx || !kept || !aligned(scores, 16) || !aligned(idx, 4) || !aligned(kept, 4))
         return TRI_ERR_INVALID;
     if (desc->S == 0) return TRI_OK;
     EvictParams e = make_evict_params(desc);
@@ -266,6 +304,10 @@ tri_status tri_compact_kv(tri_kv_desc* desc, const int32_t* idx, const int32_t* 
     e.do_select = 0;
     e.do_compact = 1;
     if ((st = cuda_status(launch_evict(e, stream))) != TRI_OK) return st;
+    MoveParams mv = make_move_params(desc, idx, budget);
+    mv.lens = desc->seq_len;
+    mv.kept = kept;
+    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream))) != TRI_OK) return st;
     FinalizeParams f{};
     f.seq_len = desc->seq_len;
     f.kept = kept;
@@ -289,7 +331,7 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     if ((st = check_budget(budget, window)) != TRI_OK) return st;
     if (!freed_ids || !freed_count || !aligned(freed_ids, 4) || !aligned(freed_count, 4)) return TRI_ERR_INVALID;
     if (idx_out && !aligned(idx_out, 4)) return TRI_ERR_INVALID;
-    if ((st = check_workspace(desc, workspace, ws_bytes)) != TRI_OK) return st;
+    if ((st = check_workspace(desc, workspace, ws_bytes, budget)) != TRI_OK) return st;
     if (events) record(events->start, stream);
     if (desc->S == 0) {
         st = cuda_status(cudaMemsetAsync(freed_count, 0, sizeof(int32_t), stream));
@@ -301,7 +343,7 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
         return st;
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const WsLayout w = ws_layout(desc);
+    const WsLayout w = ws_layout(desc, budget);
     QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
                                       reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
     q.do_plan = 1;
@@ -310,6 +352,9 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
     q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
     q.freed_count = freed_count;
+    q.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
+    q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
+    q.zero_words = reinterpret_cast<int32_t*>(ws + w.words);
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     if (events) record(events->after_query, stream);
 
@@ -321,16 +366,35 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
 
     EvictParams e = make_evict_params(desc);
     e.scores = scores;
+    e.unit_kmin = reinterpret_cast<const uint32_t*>(ws + w.kmin);
+    e.unit_kmax = reinterpret_cast<const uint32_t*>(ws + w.kmax);
     e.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
     e.budget = budget;
     e.window = window;
-    e.idx_out = idx_out;
+    e.idx_out = reinterpret_cast<int32_t*>(ws + w.idx);
+    e.idx_copy = idx_out;
     e.do_select = 1;
     e.do_compact = 1;
     e.seq_len_out = desc->seq_len;
     e.freed_off = reinterpret_cast<const int32_t*>(ws + w.freed_off);
     e.freed_ids = freed_ids;
+    e.scratch_used = reinterpret_cast<int32_t*>(ws + w.words);
+    e.unit_info = reinterpret_cast<int32_t*>(ws + w.info);
+    e.scratch_owner = reinterpret_cast<int32_t*>(ws + w.owner);
+    e.scratch_rows = w.scratch_rows;
     if ((st = cuda_status(launch_evict(e, stream))) != TRI_OK) return st;
+    MoveParams mv = make_move_params(desc, reinterpret_cast<const int32_t*>(ws + w.idx), budget);
+    mv.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
+    mv.kept = nullptr;
+    mv.unit_info = reinterpret_cast<const int32_t*>(ws + w.info);
+    mv.scratch = ws + w.scratch;
+    mv.scratch_owner = reinterpret_cast<const int32_t*>(ws + w.owner);
+    mv.scratch_used = reinterpret_cast<const int32_t*>(ws + w.words);
+    mv.scratch_rows = w.scratch_rows;
+    mv.copy_out = 1;
+    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream))) != TRI_OK) return st;
+    mv.copy_out = 0;
+    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream))) != TRI_OK) return st;
     if (events) record(events->after_evict, stream);
     return TRI_OK;
 }

@@ -37,6 +37,9 @@ struct QueryParams {
     int32_t* item_off;        // [S+1]
     int32_t* freed_off;       // [S+1]
     int32_t* freed_count;     // [1] or null
+    uint32_t* unit_kmin;      // [U] set to the largest key (min accumulator) or null
+    uint32_t* unit_kmax;      // [U] set to 0 (max accumulator) or null
+    int32_t* zero_words;      // [2] set to 0 by the plan CTA, or null
     int32_t* status;
 };
 cudaError_t launch_query(const QueryParams& p, cudaStream_t stream);
@@ -51,6 +54,8 @@ struct ScoreParams {
     const float* wts;
     float* scores;
     int64_t score_stride;     // floats between units in `scores`
+    uint32_t* unit_kmin;      // [U] smallest order key of each unit's scores
+    uint32_t* unit_kmax;      // [U] largest order key of each unit's scores
     int32_t* status;
     int L, Hkv, num_blocks, S, max_blocks;
     int heads_per_tile;       // HG, divides 8 and Hkv
@@ -63,9 +68,12 @@ cudaError_t launch_score(const ScoreParams& p, int max_items, int num_sms, cudaS
 struct EvictParams {
     const float* scores;
     int64_t score_stride;
+    const uint32_t* unit_kmin; // [U] score-key range of each unit, or null
+    const uint32_t* unit_kmax;
     const int32_t* lens;       // lengths the unit works from
     int budget, window;
     int32_t* idx_out;          // [U][budget] or null
+    int32_t* idx_copy;         // [U][budget] second copy of the kept slots, or null
     int32_t* kept_out;         // [S] or null
     const int32_t* idx_in;     // [U][budget] (compaction from given indices) or null
     const int32_t* kept_in;    // [S] or null
@@ -79,8 +87,33 @@ struct EvictParams {
     const int32_t* freed_off;  // [S+1] or null
     int32_t* freed_ids;        // or null
     int32_t* status;
+    // step plans (null outside tri_compress_step)
+    int32_t* scratch_used;     // [1] rows of the scratch handed out, 0 at launch
+    int32_t* unit_info;        // [U][4]: m0, J, mode, scratch row
+    int32_t* scratch_owner;    // [2][scratch_rows]: unit and source row of each scratch row
+    int scratch_rows;          // capacity of the scratch in rows
 };
 cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream);
+
+// Phase 2 of the compaction for all units (after launch_evict's phase 1).
+struct MoveParams {
+    const int32_t* idx;        // [U][budget] kept slots, ascending
+    int budget;
+    const int32_t* lens;       // [S] lengths before the step
+    const int32_t* kept;       // [S], or null: min(len, budget) for len > budget, else untouched
+    uint8_t* k_pool;
+    uint8_t* v_pool;
+    const int32_t* block_table;
+    int L, Hkv, num_blocks, S, max_blocks;
+    int32_t* status;
+    const int32_t* unit_info;  // [U][4] m0, J, mode, scratch row (step plans) or null
+    uint8_t* scratch;          // rows of K then V (512 bytes each) or null
+    const int32_t* scratch_owner;  // [2][scratch_rows] unit and source row of each scratch row
+    const int32_t* scratch_used;   // [1] scratch rows handed out
+    int scratch_rows;
+    int copy_out;              // 1: copy at-risk sources to the scratch; 0: move rows
+};
+cudaError_t launch_move(const MoveParams& p, int num_sms, cudaStream_t stream);
 
 // Freed-block list + new lengths after a standalone compaction.
 struct FinalizeParams {

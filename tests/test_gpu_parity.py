@@ -140,15 +140,18 @@ def _score_fill(rng, n, kind):
         return z
     if kind == "wide":
         return (rng.normal(size=n) * np.exp(rng.normal(size=n) * 20)).astype(np.float32)
+    if kind == "dups":            # spread range, many exact duplicates near every value
+        return (np.round(rng.normal(size=n) * 100) / 100).astype(np.float32)
     raise ValueError(kind)
 
 
 @pytest.mark.parametrize("budget,window", [(64, 8), (1, 0), (1, 1), (64, 64), (64, 0), (2048, 128)])
 def test_select_bit_exact_on_same_scores(budget, window):
     rng = np.random.default_rng(budget * 131 + window)
-    lens = [0, 1, budget, budget + 1, 3 * budget + 5, 40000, 777, 5000]
-    kinds = ["normal", "ties", "zeros", "wide"]
-    S, L, Hkv = len(lens), 1, 4
+    # 140000 candidates exceed the shared-memory bitmaps: streaming path
+    lens = [0, 1, budget, budget + 1, 3 * budget + 5, 40000, 777, 5000, 140000]
+    kinds = ["normal", "ties", "zeros", "wide", "dups"]
+    S, L, Hkv = len(lens), 1, len(kinds)
     max_blocks = -(-max(lens) // 16)
     k = torch.zeros(1, 1, Hkv, 16, 128, dtype=torch.bfloat16, device=DEV)
     table = torch.zeros(S, max_blocks, dtype=torch.int32, device=DEV)
