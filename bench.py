@@ -240,7 +240,8 @@ def run_ours(args, world, rank, local, dist):
         cfg = cfg.replace(L=args.layers, name=f"{cfg.name} (L={args.layers})")
     if args.workload == "cfg3":
         raise SystemExit("the decode-loop workload is measured by tests/test_gpu_workloads.py, not here")
-    wl = make_workload(cfg, device=dev, seed=rank)
+    from rope_aware_kv_tri_b200.sharding import reduce_job, shard_seed, keys_per_second
+    wl = make_workload(cfg, device=dev, seed=shard_seed(cfg.seed, rank) if world > 1 else cfg.seed)
     L, Hkv, G, Hq, S = cfg.L, cfg.Hkv, cfg.G, cfg.Hq, cfg.S
     B, W = cfg.budget, cfg.window
     stream = torch.cuda.current_stream(dev)
@@ -322,12 +323,8 @@ def run_ours(args, world, rank, local, dist):
     query_ms = [e[0].elapsed_time(e[1]) for e in evs]
     score_ms = [e[1].elapsed_time(e[2]) for e in evs]
     evict_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * keys_per_step * args.steps / (total_ms / 1e3)
+    total_ms, job_keys, job_freed = reduce_job(dist, sum(step_ms), keys_per_step, freed_per_step, dev)
+    value = keys_per_second(job_keys, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     peak, peak_kind = measured_peak()
@@ -368,7 +365,7 @@ def run_ours(args, world, rank, local, dist):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "seq_lens": lens,
                    "budget": B, "window": W, "rope_base": cfg.base, "deltas": wl.deltas,
-                   "keys_per_step_per_gpu": keys_per_step, "freed_blocks_per_step": freed_per_step,
+                   "keys_per_step_per_gpu": keys_per_step, "freed_blocks_per_step": job_freed,
                    "parallelism": f"units sharded: one independent cache per GPU x{world}",
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
                    "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
@@ -420,13 +417,10 @@ def run_e2e(args, tri, cache, wl, cfg, qbar, qabs, R, ws, freed, count, save_k, 
             times.append(a.elapsed_time(b))
     if tri.tri_sync_status(cache.status) != tri.TRI_OK:
         raise RuntimeError("device status flag raised during the end-to-end steps")
-    total = sum(times)
-    if dist is not None:
-        t = torch.tensor([total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
+    from rope_aware_kv_tri_b200.sharding import reduce_job, keys_per_second
+    total, job_keys, _ = reduce_job(dist, sum(times), keys_per_step, 0, dev)
     del host
-    return {"value": round(world * keys_per_step * len(times) / (total / 1e3), 1), "unit": UNIT,
+    return {"value": round(keys_per_second(job_keys, len(times), total), 1), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": len(times),
             "ms_per_step": round(total / len(times), 3)}
 

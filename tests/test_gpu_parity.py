@@ -321,3 +321,46 @@ def test_sequence_longer_than_its_table_is_flagged():
     out = run_step(wl, stats, 512, 64)
     assert out["status"] == tri.TRI_ERR_DEVICE_BOUNDS
     assert torch.equal(k0, wl.k_pool)
+
+
+def test_compress_step_prefix_heavy_units_mix_scratch_and_in_place():
+    """Scores that fall with the slot make almost every kept source lie below
+    the budget, so each unit's at-risk prefix is nearly B rows: the step's
+    scratch (a quarter of the kept rows) fills up and later units compact
+    their prefix in place.  Both paths must give the oracle's result."""
+    cfg = CONFIGS["cfg2"].replace(L=1, Hkv=4, G=2, lens=[700, 650], budget=256, window=16, n_samples=64,
+                                  table="shuffled")
+    wl = make_workload(cfg, device=DEV, seed=7)
+    L, Hkv, Hq = cfg.L, cfg.Hkv, cfg.Hq
+    table = wl.block_table.cpu().tolist()
+    gen = torch.Generator(device=DEV).manual_seed(3)
+    for s, n in enumerate(cfg.lens):
+        t = torch.arange(n, device=DEV, dtype=torch.float32)
+        scale = 1.0 / (1.0 + t / 50.0)
+        scale[0] = 1e-3                                  # slot 0 is evicted: every row moves
+        for l in range(L):
+            for h in range(Hkv):
+                rows = torch.randn(n, 128, device=DEV, generator=gen) * scale[:, None]
+                blocks = torch.tensor(table[s][: -(-n // 16)], device=DEV, dtype=torch.long)
+                padded = torch.zeros(len(blocks) * 16, 128, device=DEV)
+                padded[:n] = rows
+                wl.k_pool[l, blocks, h] = padded.view(len(blocks), 16, 128).to(torch.bfloat16)
+    # norm-only scoring: qbar = 0, E|q_i| = 1, R = 0
+    stats = (torch.zeros(L, Hq, 128, device=DEV), torch.ones(L, Hq, 64, device=DEV), torch.zeros(L, Hq, device=DEV))
+    ref_stats = tuple(x.double().cpu().numpy() for x in stats)
+    lens = list(cfg.lens)
+    kept = [min(n, cfg.budget) for n in lens]
+    pk, pv = wl.k_pool.clone(), wl.v_pool.clone()
+    out = run_step(wl, stats, cfg.budget, cfg.window)
+    assert out["status"] == tri.TRI_OK
+    idx = out["idx"]
+    assert out["freed"] == freed_expected(wl.block_table, lens, kept)
+    for s, n in enumerate(lens):
+        for l in range(L):
+            for h in range(Hkv):
+                ref = oracle_unit_scores(wl, unit_rows(pk, table[s], n, l, h), ref_stats, s, l, h)
+                check_selection(idx[s, l, h].cpu().numpy(), ref, n, cfg.budget, cfg.window)
+                assert int((idx[s, l, h] < cfg.budget).sum()) > cfg.budget // 2     # prefix-heavy indeed
+    ek, ev = expected_pools_after(pk, pv, wl.block_table, lens, idx, kept)
+    assert torch.equal(wl.k_pool.view(torch.int16), ek.view(torch.int16))
+    assert torch.equal(wl.v_pool.view(torch.int16), ev.view(torch.int16))
