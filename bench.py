@@ -303,7 +303,9 @@ def run_ours(args, world, rank, local, dist):
     if dist is not None:
         dist.barrier()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # Timed steps: one event pair around each tri_compress_step (its kernels
+    # then overlap their launches programmatically).
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     clocks = ClockSampler(local)
     clocks.start()
     torch.cuda.synchronize(dev)
@@ -311,18 +313,28 @@ def run_ours(args, world, rank, local, dist):
         dist.barrier()
     for k in range(args.steps):
         restore()
-        step(events=evs[k])
+        evs[k][0].record()
+        step()
+        evs[k][1].record()
     torch.cuda.synchronize(dev)
     if dist is not None:
         dist.barrier()
     clocks.stop()
     if tri.tri_sync_status(cache.status) != tri.TRI_OK:
         raise RuntimeError("device status flag raised during the timed steps")
+    step_ms = [e[0].elapsed_time(e[1]) for e in evs]
 
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    query_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    score_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    evict_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    # Phase times (live, same workload): the library records events between
+    # its kernels, which serialises their launches, so this is a separate loop.
+    n_phase = min(args.steps, 200)
+    pevs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n_phase)]
+    for k in range(n_phase):
+        restore()
+        step(events=pevs[k])
+    torch.cuda.synchronize(dev)
+    query_ms = [e[0].elapsed_time(e[1]) for e in pevs]
+    score_ms = [e[1].elapsed_time(e[2]) for e in pevs]
+    evict_ms = [e[2].elapsed_time(e[3]) for e in pevs]
     total_ms, job_keys, job_freed = reduce_job(dist, sum(step_ms), keys_per_step, freed_per_step, dev)
     value = keys_per_second(job_keys, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
@@ -338,12 +350,13 @@ def run_ours(args, world, rank, local, dist):
                 "kernel": "score_kernel", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s",
                 "algorithmic_bytes_per_launch": k_bytes, "ms_per_launch": round(score_mean, 5),
+                "timing": f"CUDA events around the score kernel, {n_phase} live steps",
                 "nominal_hbm_gbs": NOMINAL_HBM_GBS}
     step_bytes = k_bytes + moved_bytes
     step_achieved = step_bytes / (ms_per_step / 1e3) / 1e9
     step_roofline = {"bound": "hbm", "achieved": round(step_achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(step_achieved / peak, 4), "bytes_per_step": step_bytes,
-                     "moved_rows": moved, "phase_ms": {"query": round(statistics.mean(query_ms), 5),
+                     "moved_rows": moved, "phase_ms_serialised": {"query": round(statistics.mean(query_ms), 5),
                                                        "score": round(score_mean, 5),
                                                        "select_compact": round(statistics.mean(evict_ms), 5)}}
 
@@ -369,7 +382,8 @@ def run_ours(args, world, rank, local, dist):
                    "parallelism": f"units sharded: one independent cache per GPU x{world}",
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
                    "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
-                   "timing": "CUDA events around each tri_compress_step; kept-region restore untimed"},
+                   "timing": "CUDA events around each tri_compress_step; kept-region restore and L2 flush "
+                             "untimed; per-phase times from a separate live loop with phase events"},
         "roofline": roofline, "step_roofline": step_roofline,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 5 * args.steps, "clocks": clk,
     }

@@ -63,6 +63,8 @@ constexpr int kListCap = 4096;                    // boundary-bucket pairs kept 
 constexpr int kBitmapWords = 4096;                // bitmaps of up to 131072 candidate slots
 constexpr int kLinBins = 4096;                    // linear buckets over a unit's score range
 constexpr int kRankListMax = 1024;                // lists up to this size are ranked directly
+constexpr int kCodeSlots = 32768;                 // candidates whose buckets fit in shared memory
+constexpr int kOneListCap = 1024;                 // cut-bucket entries in the one-pass layout
 constexpr int kUnroll = 8;                        // 16-byte loads in flight per thread in a walk
 constexpr int kStep = 128;                        // slots per warp step (4 per lane)
 constexpr int kRowBytes = kHeadDim * 2;           // 256
@@ -72,17 +74,35 @@ constexpr int kModeInPlace = 0, kModeScratch = 1;  // how a unit's rows [m0, J) 
 constexpr int kMoveThreads = 256;
 constexpr int kMoveRows = 8;                      // rows in flight per warp in move_kernel
 
-struct SelectScratch {
+// Shared scratch of the selection, in one of two layouts.  "two" serves
+// units with more candidates than `code` holds (two streaming passes);
+// "one" keeps every candidate's linear bucket in shared memory so the
+// scores are streamed once.  Both start with the histogram.
+struct TwoPassScratch {
     int hist[kTopBins];
     uint32_t list_key[kListCap];
     int list_slot[kListCap];
     uint32_t gt_bits[kBitmapWords];   // candidates kept for a score above the cut
     uint32_t eq_bits[kBitmapWords];   // candidates whose score equals the cut
 };
+struct OnePassScratch {
+    int hist[kLinBins];
+    uint32_t gt_bits[kCodeSlots / 32];
+    uint32_t eq_bits[kCodeSlots / 32];
+    uint32_t list_key[kOneListCap];
+    int list_slot[kOneListCap];
+    uint16_t code[kCodeSlots];        // linear bucket of every candidate
+};
+union SelectScratch {
+    TwoPassScratch two;
+    OnePassScratch one;
+    int hist[kTopBins];
+};
 struct EvictSmem {
     union {
         SelectScratch sel;
     } u;
+    static_assert(sizeof(OnePassScratch) <= 100 * 1024, "one-pass scratch too large");
     int warp_a[kEvictWarps];      // keys > thr in the segment (part 1)
     int warp_b[kEvictWarps];      // keys == thr in the segment
     int warp_c[kEvictWarps];      // keys > thr in the segment (part 2)
@@ -241,13 +261,173 @@ __device__ __forceinline__ int lin_bucket(float x, float lo, float scale) {
     return b < 0 ? 0 : (b > kLinBins - 1 ? kLinBins - 1 : b);
 }
 
+// The cut from the list of the cut bucket's keys (rem = the cut's rank in
+// the bucket), then the kept candidates from the bitmaps: gt_bits holds the
+// candidates above the bucket; the list's keys above the cut join them, the
+// ones equal to it go to eq_bits, of which the first need_eq in slot order
+// are kept.  Emits the take kept slots ascending into sidx.
+__device__ void finish_from_list(const uint32_t* list_key, const int* list_slot, int n, int rem, uint32_t* gt_bits,
+                                 uint32_t* eq_bits, int nwords, int take, int* sidx, int* hist, EvictSmem& sm) {
+    uint32_t thr;
+    int need_eq;
+    if (n <= kRankListMax) {
+        // the cut key is the list key with (#greater) < rem <= (#greater-or-equal)
+        for (int i = threadIdx.x; i < n; i += kEvictThreads) {
+            const uint32_t key = list_key[i];
+            int gt = 0, ge = 0;
+            for (int k = 0; k < n; ++k) {
+                const uint32_t o = list_key[k];
+                gt += o > key ? 1 : 0;
+                ge += o >= key ? 1 : 0;
+            }
+            if (gt < rem && rem <= ge) {         // every thread that finds it writes the same values
+                sm.bcast[2] = (int)key;
+                sm.bcast[3] = rem - gt;
+            }
+        }
+        __syncthreads();
+        thr = (uint32_t)sm.bcast[2];
+        need_eq = sm.bcast[3];
+    } else {
+        uint32_t prefix = 0, mask = 0;
+        list_radix_pass(list_key, n, prefix, mask, rem, 21, 11, hist, sm);
+        list_radix_pass(list_key, n, prefix, mask, rem, 10, 11, hist, sm);
+        list_radix_pass(list_key, n, prefix, mask, rem, 0, 10, hist, sm);
+        thr = prefix;
+        need_eq = rem;
+    }
+    for (int i = threadIdx.x; i < n; i += kEvictThreads) {
+        const uint32_t key = list_key[i];
+        const int t = list_slot[i];
+        if (key > thr) atomicOr(&gt_bits[t >> 5], 1u << (t & 31));
+        else if (key == thr) atomicOr(&eq_bits[t >> 5], 1u << (t & 31));
+    }
+    __syncthreads();
+    // Emission: each thread owns a run of words; the first need_eq tied
+    // candidates in slot order are kept.
+    const int wpt = (nwords + kEvictThreads - 1) / kEvictThreads;
+    const int w0 = min(threadIdx.x * wpt, nwords), w1 = min(w0 + wpt, nwords);
+    int my_eq = 0;
+    for (int w = w0; w < w1; ++w) my_eq += __popc(eq_bits[w]);
+    int tot;
+    int eq_before = block_exclusive_scan<kEvictThreads>(my_eq, sm.scan_tmp, tot);
+    int my_keep = 0;
+    for (int w = w0; w < w1; ++w) {
+        uint32_t e = eq_bits[w];
+        int allow = need_eq - eq_before;
+        eq_before += __popc(e);
+        uint32_t keep_e = 0u;
+        while (e && allow > 0) {
+            const uint32_t low = e & (0u - e);
+            keep_e |= low;
+            e ^= low;
+            --allow;
+        }
+        const uint32_t kw = gt_bits[w] | keep_e;
+        gt_bits[w] = kw;
+        my_keep += __popc(kw);
+    }
+    int off = block_exclusive_scan<kEvictThreads>(my_keep, sm.scan_tmp, tot);
+    for (int w = w0; w < w1; ++w) {
+        uint32_t kw = gt_bits[w];
+        while (kw) {
+            const int b = __ffs(kw) - 1;
+            if (off < take) sidx[off] = w * 32 + b;
+            ++off;
+            kw &= kw - 1u;
+        }
+    }
+    __syncthreads();
+}
+
+// One streaming pass (cand <= kCodeSlots): the histogram pass also keeps
+// every candidate's linear bucket in shared memory; the bitmap of buckets
+// above the cut's and the cut bucket's slots then come from shared memory,
+// and only the (few) cut-bucket scores are read again.
+__device__ bool select_one_pass(const float* __restrict__ sc, int cand, int take, float lo, float scale, int* sidx,
+                                EvictSmem& sm) {
+    OnePassScratch& o = sm.u.sel.one;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kLinBins; i += kEvictThreads) o.hist[i] = 0;
+    __syncthreads();
+    const int nvec = cand >> 2;
+    const float4* v4 = reinterpret_cast<const float4*>(sc);
+    for (int v0 = threadIdx.x; v0 < nvec; v0 += kEvictThreads * kUnroll) {
+        float4 x[kUnroll];
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const int v = v0 + k * kEvictThreads;
+            x[k] = v < nvec ? v4[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int k = 0; k < kUnroll; ++k) {
+            const int v = v0 + k * kEvictThreads;
+            if (v < nvec) {
+                const int b0 = lin_bucket(x[k].x, lo, scale), b1 = lin_bucket(x[k].y, lo, scale);
+                const int b2 = lin_bucket(x[k].z, lo, scale), b3 = lin_bucket(x[k].w, lo, scale);
+                *reinterpret_cast<uint2*>(&o.code[4 * v]) =
+                    make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
+                atomicAdd(&o.hist[b0], 1);
+                atomicAdd(&o.hist[b1], 1);
+                atomicAdd(&o.hist[b2], 1);
+                atomicAdd(&o.hist[b3], 1);
+            }
+        }
+    }
+    for (int t = 4 * nvec + threadIdx.x; t < cand; t += kEvictThreads) {
+        const int b = lin_bucket(sc[t], lo, scale);
+        o.code[t] = (uint16_t)b;
+        atomicAdd(&o.hist[b], 1);
+    }
+    __syncthreads();
+    int rem = take;
+    const int bstar = pick_bin(o.hist, kLinBins, rem, sm);
+    if (o.hist[bstar] > kOneListCap) return false;
+    const int nwords = (cand + 31) / 32;
+    for (int w = threadIdx.x; w < nwords; w += kEvictThreads) o.eq_bits[w] = 0u;
+    if (threadIdx.x == 0) sm.n_list = 0;
+    __syncthreads();
+    // 8 buckets per 16-byte load; 4 lanes make one 32-slot word
+    const int nq = (cand + 7) / 8;
+    for (int q0 = warp * 32; q0 < nq; q0 += kEvictWarps * 32) {
+        const int q = q0 + lane;
+        uint32_t m = 0u;
+        if (q < nq) {
+            const uint4 c4 = *reinterpret_cast<const uint4*>(&o.code[8 * q]);
+            const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int t = 8 * q + i;
+                const int b = (int)((cw[i >> 1] >> (16 * (i & 1))) & 0xffffu);
+                if (t < cand) {
+                    if (b > bstar) m |= 1u << i;
+                    else if (b == bstar) {
+                        const int pos = atomicAdd(&sm.n_list, 1);
+                        if (pos < kOneListCap) o.list_slot[pos] = t;
+                    }
+                }
+            }
+        }
+        uint32_t word = m << (8 * (lane & 3));
+        word |= __shfl_xor_sync(0xffffffffu, word, 1);
+        word |= __shfl_xor_sync(0xffffffffu, word, 2);
+        if ((lane & 3) == 0 && q < nq) o.gt_bits[q >> 2] = word;
+    }
+    __syncthreads();
+    const int n = min(sm.n_list, kOneListCap);
+    for (int i = threadIdx.x; i < n; i += kEvictThreads) o.list_key[i] = order_key(sc[o.list_slot[i]]);
+    __syncthreads();
+    finish_from_list(o.list_key, o.list_slot, n, rem, o.gt_bits, o.eq_bits, nwords, take, sidx, o.hist, sm);
+    return true;
+}
+
 // Selection over a known score range [kmin, kmax] (order keys): a linear
-// histogram finds the bucket of the cut; one more walk marks the candidates
-// above that bucket in a bitmap and lists the bucket's (key, slot) pairs;
-// the exact cut key and its tie count come from radix passes over the list;
-// the kept slots are then emitted from the bitmaps in slot order.  Returns
-// false, with nothing written, when the range is not finite, the candidates
-// exceed the bitmap, or the cut's bucket exceeds the list.
+// histogram finds the bucket of the cut; the candidates above that bucket go
+// to a bitmap and the bucket's (key, slot) pairs to a list; the exact cut
+// key and its tie count come from the list; the kept slots are then emitted
+// from the bitmaps in slot order.  Returns false, with nothing kept, when the
+// range is not finite, the candidates exceed the bitmap, or the cut's
+// bucket exceeds the list.
 __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, uint32_t kmin, uint32_t kmax,
                               int* sidx, EvictSmem& sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -261,6 +441,7 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
         return true;
     }
     const float scale = (float)(kLinBins - 1) / span;
+    if (cand <= kCodeSlots) return select_one_pass(sc, cand, take, lo, scale, sidx, sm);
     int* hist = sm.u.sel.hist;
     // warp segments of whole 128-slot steps
     const int seg = ((cand + kEvictWarps - 1) / kEvictWarps + kStep - 1) / kStep * kStep;
@@ -300,7 +481,7 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
 
     // Pass 2: bitmap of candidates above the cut's bucket; list of the bucket.
     const int nwords = (cand + 31) / 32;
-    for (int w = threadIdx.x; w < nwords; w += kEvictThreads) sm.u.sel.eq_bits[w] = 0u;
+    for (int w = threadIdx.x; w < nwords; w += kEvictThreads) sm.u.sel.two.eq_bits[w] = 0u;
     if (threadIdx.x == 0) sm.n_list = 0;
     __syncthreads();
     const uint32_t lt = lanemask_lt();
@@ -323,7 +504,7 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
                     inb[c] = __ballot_sync(0xffffffffu, valid && b == bstar);
                     n_in += __popc(inb[c]);
                 }
-                if (lane < 4 && base + 32 * lane < end) sm.u.sel.gt_bits[(base >> 5) + lane] = step_word(above, lane);
+                if (lane < 4 && base + 32 * lane < end) sm.u.sel.two.gt_bits[(base >> 5) + lane] = step_word(above, lane);
                 if (n_in) {
                     int at = 0;
                     if (lane == 0) at = atomicAdd(&sm.n_list, n_in);
@@ -333,8 +514,8 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
                         if (inb[c] & (1u << lane)) {
                             const int pos = at + __popc(inb[c] & lt);
                             if (pos < kListCap) {
-                                sm.u.sel.list_key[pos] = order_key(x[k][c]);
-                                sm.u.sel.list_slot[pos] = t + c;
+                                sm.u.sel.two.list_key[pos] = order_key(x[k][c]);
+                                sm.u.sel.two.list_slot[pos] = t + c;
                             }
                         }
                         at += __popc(inb[c]);
@@ -345,76 +526,8 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
     }
     __syncthreads();
     const int n = min(sm.n_list, kListCap);
-    uint32_t thr;
-    int need_eq;
-    if (n <= kRankListMax) {
-        // the cut key is the list key with (#greater) < rem <= (#greater-or-equal)
-        for (int i = threadIdx.x; i < n; i += kEvictThreads) {
-            const uint32_t key = sm.u.sel.list_key[i];
-            int gt = 0, ge = 0;
-            for (int k = 0; k < n; ++k) {
-                const uint32_t o = sm.u.sel.list_key[k];
-                gt += o > key ? 1 : 0;
-                ge += o >= key ? 1 : 0;
-            }
-            if (gt < rem && rem <= ge) {         // every thread that finds it writes the same values
-                sm.bcast[2] = (int)key;
-                sm.bcast[3] = rem - gt;
-            }
-        }
-        __syncthreads();
-        thr = (uint32_t)sm.bcast[2];
-        need_eq = sm.bcast[3];
-    } else {
-        uint32_t prefix = 0, mask = 0;
-        list_radix_pass(sm.u.sel.list_key, n, prefix, mask, rem, 21, 11, hist, sm);
-        list_radix_pass(sm.u.sel.list_key, n, prefix, mask, rem, 10, 11, hist, sm);
-        list_radix_pass(sm.u.sel.list_key, n, prefix, mask, rem, 0, 10, hist, sm);
-        thr = prefix;
-        need_eq = rem;
-    }
-    for (int i = threadIdx.x; i < n; i += kEvictThreads) {
-        const uint32_t key = sm.u.sel.list_key[i];
-        const int t = sm.u.sel.list_slot[i];
-        if (key > thr) atomicOr(&sm.u.sel.gt_bits[t >> 5], 1u << (t & 31));
-        else if (key == thr) atomicOr(&sm.u.sel.eq_bits[t >> 5], 1u << (t & 31));
-    }
-    __syncthreads();
-    // Emission: each thread owns a run of words; the first need_eq tied
-    // candidates in slot order are kept.
-    const int wpt = (nwords + kEvictThreads - 1) / kEvictThreads;
-    const int w0 = min(threadIdx.x * wpt, nwords), w1 = min(w0 + wpt, nwords);
-    int my_eq = 0;
-    for (int w = w0; w < w1; ++w) my_eq += __popc(sm.u.sel.eq_bits[w]);
-    int tot;
-    int eq_before = block_exclusive_scan<kEvictThreads>(my_eq, sm.scan_tmp, tot);
-    int my_keep = 0;
-    for (int w = w0; w < w1; ++w) {
-        uint32_t e = sm.u.sel.eq_bits[w];
-        int allow = need_eq - eq_before;
-        eq_before += __popc(e);
-        uint32_t keep_e = 0u;
-        while (e && allow > 0) {
-            const uint32_t low = e & (0u - e);
-            keep_e |= low;
-            e ^= low;
-            --allow;
-        }
-        const uint32_t kw = sm.u.sel.gt_bits[w] | keep_e;
-        sm.u.sel.gt_bits[w] = kw;
-        my_keep += __popc(kw);
-    }
-    int off = block_exclusive_scan<kEvictThreads>(my_keep, sm.scan_tmp, tot);
-    for (int w = w0; w < w1; ++w) {
-        uint32_t kw = sm.u.sel.gt_bits[w];
-        while (kw) {
-            const int b = __ffs(kw) - 1;
-            if (off < take) sidx[off] = w * 32 + b;
-            ++off;
-            kw &= kw - 1u;
-        }
-    }
-    __syncthreads();
+    finish_from_list(sm.u.sel.two.list_key, sm.u.sel.two.list_slot, n, rem, sm.u.sel.two.gt_bits,
+                     sm.u.sel.two.eq_bits, nwords, take, sidx, hist, sm);
     return true;
 }
 
@@ -511,8 +624,8 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
                             if (d == top) {
                                 const int pos = atomicAdd(&sm.n_list, 1);
                                 if (pos < kListCap) {
-                                    sm.u.sel.list_key[pos] = key;
-                                    sm.u.sel.list_slot[pos] = t;
+                                    sm.u.sel.two.list_key[pos] = key;
+                                    sm.u.sel.two.list_slot[pos] = t;
                                 }
                             }
                         }
@@ -523,16 +636,16 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
             if (lane == 0) sm.warp_a[warp] = above;
             __syncthreads();
             const int n = min(sm.n_list, kListCap);
-            list_radix_pass(sm.u.sel.list_key, n, prefix, mask, rem, 10, 10, hist, sm);
-            list_radix_pass(sm.u.sel.list_key, n, prefix, mask, rem, 0, 10, hist, sm);
+            list_radix_pass(sm.u.sel.two.list_key, n, prefix, mask, rem, 10, 10, hist, sm);
+            list_radix_pass(sm.u.sel.two.list_key, n, prefix, mask, rem, 0, 10, hist, sm);
             if (threadIdx.x < kEvictWarps) {
                 sm.warp_b[threadIdx.x] = 0;
                 sm.warp_c[threadIdx.x] = 0;
             }
             __syncthreads();
             for (int i = threadIdx.x; i < n; i += kEvictThreads) {
-                const uint32_t key = sm.u.sel.list_key[i];
-                const int w = sm.u.sel.list_slot[i] / seg;
+                const uint32_t key = sm.u.sel.two.list_key[i];
+                const int w = sm.u.sel.two.list_slot[i] / seg;
                 if (key > prefix) atomicAdd(&sm.warp_c[w], 1);
                 else if (key == prefix) atomicAdd(&sm.warp_b[w], 1);
             }
@@ -701,6 +814,7 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
     const int LH = p.L * p.Hkv;
     const int s = u / LH, rem = u % LH, l = rem / p.Hkv, h = rem % p.Hkv;
     const bool head0 = (l == 0 && h == 0);
+    wait_prior_grid();
     int len = p.lens[s];
     if (len < 0 || (int64_t)len > (int64_t)p.max_blocks * kBlockRows) {
         if (threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
@@ -867,6 +981,7 @@ __device__ void copy_out_rows(const MoveParams& p) {
 }
 
 __global__ void __launch_bounds__(kMoveThreads, 3) move_kernel(const MoveParams p) {
+    wait_prior_grid();
     if (p.copy_out) {
         copy_out_rows(p);
         return;
@@ -1004,25 +1119,23 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
 
 }  // namespace
 
-cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream) {
+cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream, bool pdl) {
     const int U = p.S * p.L * p.Hkv;
     if (U == 0) return cudaSuccess;
     const size_t smem = sizeof(EvictSmem) + (size_t)p.budget * sizeof(int);
     cudaError_t e = cudaFuncSetAttribute(evict_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    evict_kernel<<<U, kEvictThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(evict_kernel, dim3(U), dim3(kEvictThreads), smem, stream, pdl, p);
 }
 
-cudaError_t launch_move(const MoveParams& p, int num_sms, cudaStream_t stream) {
+cudaError_t launch_move(const MoveParams& p, int num_sms, cudaStream_t stream, bool pdl) {
     const int64_t tiles = p.copy_out ? ((int64_t)p.scratch_rows + kMoveRows - 1) / kMoveRows
                                      : (int64_t)p.S * p.L * p.Hkv * ((p.budget + 31) / 32);
     if (tiles == 0) return cudaSuccess;
     if (tiles > INT_MAX) return cudaErrorInvalidValue;
     int64_t grid = (tiles + kMoveThreads / 32 - 1) / (kMoveThreads / 32);
     if (grid > (int64_t)num_sms * 3) grid = (int64_t)num_sms * 3;
-    move_kernel<<<(int)grid, kMoveThreads, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(move_kernel, dim3((unsigned)grid), dim3(kMoveThreads), 0, stream, pdl, p);
 }
 
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t stream) {

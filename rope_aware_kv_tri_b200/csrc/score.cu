@@ -257,6 +257,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
         fence_mbar_init();
     }
     __syncthreads();
+    wait_prior_grid();          // the folded queries and the plan come from query_kernel
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == kConsumerWarps) {
         if (lane == 0) produce(p, tiles, full, empty, meta, abort_flag);
@@ -278,7 +279,7 @@ int score_heads_per_tile(int Hkv) {
     return 1;
 }
 
-cudaError_t launch_score(const ScoreParams& p_in, int max_items, int num_sms, cudaStream_t stream) {
+cudaError_t launch_score(const ScoreParams& p_in, int max_items, int num_sms, cudaStream_t stream, bool pdl) {
     ScoreParams p = p_in;
     int stages = kStageBudgetBytes / (p.heads_per_tile * kTileBytes);
     if (stages > kMaxStages) stages = kMaxStages;
@@ -290,8 +291,7 @@ cudaError_t launch_score(const ScoreParams& p_in, int max_items, int num_sms, cu
     int grid = num_sms * 2;
     if (max_items < grid) grid = max_items;
     if (grid < 1) grid = 1;
-    score_kernel<<<grid, kScoreThreads, smem, stream>>>(p);
-    return cudaGetLastError();
+    return launch_kernel(score_kernel, dim3(grid), dim3(kScoreThreads), smem, stream, pdl, p);
 }
 
 }  // namespace tri

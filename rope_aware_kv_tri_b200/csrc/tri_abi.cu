@@ -358,9 +358,12 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     if (events) record(events->after_query, stream);
 
+    // Later kernels overlap their launch with the previous one's tail unless
+    // phase events sit between them.
+    const bool pdl = events == nullptr;
     float* scores = reinterpret_cast<float*>(ws + w.scores);
     ScoreParams sp = make_score_params(desc, ws, w, scores, (int64_t)desc->max_blocks * kBlockRows);
-    if ((st = cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream))) != TRI_OK)
+    if ((st = cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream, pdl))) != TRI_OK)
         return st;
     if (events) record(events->after_score, stream);
 
@@ -382,7 +385,7 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     e.unit_info = reinterpret_cast<int32_t*>(ws + w.info);
     e.scratch_owner = reinterpret_cast<int32_t*>(ws + w.owner);
     e.scratch_rows = w.scratch_rows;
-    if ((st = cuda_status(launch_evict(e, stream))) != TRI_OK) return st;
+    if ((st = cuda_status(launch_evict(e, stream, pdl))) != TRI_OK) return st;
     MoveParams mv = make_move_params(desc, reinterpret_cast<const int32_t*>(ws + w.idx), budget);
     mv.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
     mv.kept = nullptr;
@@ -392,9 +395,9 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     mv.scratch_used = reinterpret_cast<const int32_t*>(ws + w.words);
     mv.scratch_rows = w.scratch_rows;
     mv.copy_out = 1;
-    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream))) != TRI_OK) return st;
+    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream, pdl))) != TRI_OK) return st;
     mv.copy_out = 0;
-    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream))) != TRI_OK) return st;
+    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream, pdl))) != TRI_OK) return st;
     if (events) record(events->after_evict, stream);
     return TRI_OK;
 }

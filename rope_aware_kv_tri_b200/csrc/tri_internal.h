@@ -9,6 +9,25 @@
 
 namespace tri {
 
+// Launch `kernel` with the programmatic-serialization attribute when `pdl`
+// is set (the kernel must call wait_prior_grid before reading what earlier
+// work in the stream wrote), else as a plain launch.
+template <typename Kernel, typename Params>
+cudaError_t launch_kernel(Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t stream, bool pdl,
+                          const Params& params) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, params);
+}
+
 constexpr int kHeadDim = TRI_HEAD_DIM;          // D
 constexpr int kBands = TRI_HEAD_DIM / 2;        // n
 constexpr int kBlockRows = TRI_BLOCK_SIZE;      // rows per paged block
@@ -62,7 +81,7 @@ struct ScoreParams {
     int stages;
 };
 int score_heads_per_tile(int Hkv);
-cudaError_t launch_score(const ScoreParams& p, int max_items, int num_sms, cudaStream_t stream);
+cudaError_t launch_score(const ScoreParams& p, int max_items, int num_sms, cudaStream_t stream, bool pdl = false);
 
 // --------------------------------------------------- select + compaction
 struct EvictParams {
@@ -93,7 +112,7 @@ struct EvictParams {
     int32_t* scratch_owner;    // [2][scratch_rows]: unit and source row of each scratch row
     int scratch_rows;          // capacity of the scratch in rows
 };
-cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream);
+cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream, bool pdl = false);
 
 // Phase 2 of the compaction for all units (after launch_evict's phase 1).
 struct MoveParams {
@@ -113,7 +132,7 @@ struct MoveParams {
     int scratch_rows;
     int copy_out;              // 1: copy at-risk sources to the scratch; 0: move rows
 };
-cudaError_t launch_move(const MoveParams& p, int num_sms, cudaStream_t stream);
+cudaError_t launch_move(const MoveParams& p, int num_sms, cudaStream_t stream, bool pdl = false);
 
 // Freed-block list + new lengths after a standalone compaction.
 struct FinalizeParams {
