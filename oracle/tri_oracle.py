@@ -136,13 +136,22 @@ def head_score(keys: np.ndarray, qbar_g: np.ndarray, qabs_g: np.ndarray, R_g: fl
 
 
 def unit_scores(keys: np.ndarray, qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray,
-                p: int, deltas: Sequence[int], base: float) -> np.ndarray:
-    """Mean over the G query heads of ``head_score`` (qbar [G, D], ...)."""
+                p: int, deltas: Sequence[int], base: float, aggregate: str = "mean") -> np.ndarray:
+    """The G query heads' ``head_score`` combined per key (qbar [G, D], ...):
+    their mean (the method's reading), or their maximum (a variant)."""
     G = qbar.shape[0]
-    total = np.zeros(keys.shape[0], dtype=np.float64)
-    for g in range(G):
-        total += head_score(keys, qbar[g], qabs[g], R[g], p, deltas, base)
-    return total / G
+    per_head = [head_score(keys, qbar[g], qabs[g], R[g], p, deltas, base) for g in range(G)]
+    if aggregate == "mean":
+        total = np.zeros(keys.shape[0], dtype=np.float64)
+        for sg in per_head:
+            total += sg
+        return total / G
+    if aggregate == "max":
+        best = per_head[0].copy()
+        for sg in per_head[1:]:
+            best = np.maximum(best, sg)
+        return best
+    raise ValueError("aggregate must be 'mean' or 'max'")
 
 
 def group_query(qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray, p: int,
@@ -170,19 +179,21 @@ def group_query(qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray, p: int,
 # figure, top-K selection).
 # ----------------------------------------------------------------------------
 
-def select(scores: Sequence[float], length: int, budget: int, window: int) -> np.ndarray:
+def select(scores: Sequence[float], length: int, budget: int, window: int, sinks: int = 0) -> np.ndarray:
     """Ascending slot indices kept for one unit.
 
-    If length <= budget every slot is kept.  Otherwise the last ``window``
-    slots are kept, plus the (budget - window) best of the other slots,
-    ordered by score (higher first) and then by slot (lower first).
+    If length <= budget every slot is kept.  Otherwise the first ``sinks``
+    slots and the last ``window`` slots are kept, plus the
+    (budget - window - sinks) best of the slots between them, ordered by
+    score (higher first) and then by slot (lower first).  Sinks are the
+    optional attention-sink variant; the method itself keeps none.
     """
-    if not (budget >= 1 and 0 <= window <= budget):
-        raise ValueError("need budget >= 1 and 0 <= window <= budget")
+    if not (budget >= 1 and 0 <= window and 0 <= sinks and window + sinks <= budget):
+        raise ValueError("need budget >= 1 and 0 <= window, sinks with window + sinks <= budget")
     if length <= budget:
         return np.arange(length, dtype=np.int64)
     cand = length - window
-    take = budget - window
+    take = budget - window - sinks
 
     def rank_key(t: int):
         v = float(scores[t])
@@ -190,8 +201,8 @@ def select(scores: Sequence[float], length: int, budget: int, window: int) -> np
             v = -math.inf
         return (-v, t)
 
-    best = sorted(range(cand), key=rank_key)[:take]
-    kept = sorted(best) + list(range(cand, length))
+    best = sorted(range(sinks, cand), key=rank_key)[:take]
+    kept = list(range(sinks)) + sorted(best) + list(range(cand, length))
     return np.asarray(kept, dtype=np.int64)
 
 
@@ -257,32 +268,44 @@ def compress_unit(keys_f64: np.ndarray, k_rows: np.ndarray, v_rows: np.ndarray,
 def compress_step(k_vals: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
                   block_table: np.ndarray, seq_len: Sequence[int], cur_pos: Sequence[int],
                   qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray, G: int,
-                  deltas: Sequence[int], base: float, budget: int, window: int) -> Dict:
+                  deltas: Sequence[int], base: float, budget: int, window: int,
+                  sinks: int = 0, trigger: int = 0, aggregate: str = "mean") -> Dict:
     """One compression step over every unit of every sequence.
 
     k_vals : float64 [L][NB][Hkv][bs][D], the cached keys' values
     k_bits, v_bits : the pools in any representation; copies are returned
     qbar [L][Hq][D], qabs [L][Hq][D/2], R [L][Hq] : head statistics
 
+    A sequence is compressed only when its length exceeds ``trigger`` (which
+    defaults to the budget and is never below it); shorter sequences are left
+    as they are.
+
     Returns a dict with the new pools, new lengths, the freed block ids (in
     sequence order, each sequence's blocks in table order), and per unit
     (s, l, h) its scores and kept indices.
     """
     L, _, Hkv, bs, _ = k_vals.shape
+    trigger = max(int(trigger), int(budget))
     new_k, new_v = k_bits.copy(), v_bits.copy()
     new_len, freed = [], []
     scores, kept_idx = {}, {}
     for s, length in enumerate(seq_len):
         length = int(length)
         table_row = block_table[s]
+        if length <= trigger:
+            for l in range(L):
+                for h in range(Hkv):
+                    kept_idx[(s, l, h)] = np.arange(length, dtype=np.int64)
+            new_len.append(length)
+            continue
         kept = min(length, budget)
         for l in range(L):
             for h in range(Hkv):
                 g0 = h * G
                 keys = unit_rows(k_vals, table_row, length, l, h)
                 sc = unit_scores(keys, qbar[l, g0:g0 + G], qabs[l, g0:g0 + G], R[l, g0:g0 + G],
-                                 int(cur_pos[s]), deltas, base)
-                idx = select(sc, length, budget, window)
+                                 int(cur_pos[s]), deltas, base, aggregate)
+                idx = select(sc, length, budget, window, sinks)
                 assert idx.shape[0] == kept
                 kr = unit_rows(k_bits, table_row, length, l, h)
                 vr = unit_rows(v_bits, table_row, length, l, h)

@@ -27,6 +27,8 @@ def _all_pins():
             out += [(name, lambda fn=fn, a=a: fn(*a)) for a in [(8, 1e4, 37), (128, 5e5, 32768)]]
         elif name == "test_select_brute_force_dominance":
             out += [(name, lambda fn=fn, s=s: fn(s)) for s in range(30)]
+        elif name == "test_select_with_sinks_brute_force":
+            out += [(name, lambda fn=fn, s=s: fn(s)) for s in range(20)]
         elif len(params) == 0:
             out.append((name, fn))
     return out
@@ -39,7 +41,7 @@ def _caught(monkeypatch, attr, replacement):
     for name, fn in _all_pins():
         try:
             fn()
-        except Exception:
+        except (Exception, pytest.fail.Exception):   # a pin's pytest.raises failing counts
             failed.append(name)
     return failed
 
@@ -94,11 +96,11 @@ def _head_score_squared_norm(keys, qbar_g, qabs_g, R_g, p, deltas, base):
     return trig + (1 - R_g) * norm
 
 
-def _unit_scores_sum(keys, qbar, qabs, R, p, deltas, base):
+def _unit_scores_sum(keys, qbar, qabs, R, p, deltas, base, aggregate="mean"):
     return sum(T.head_score(keys, qbar[g], qabs[g], R[g], p, deltas, base) for g in range(qbar.shape[0]))
 
 
-def _select_ties_high(scores, length, budget, window):
+def _select_ties_high(scores, length, budget, window, sinks=0):
     if length <= budget:
         return np.arange(length)
     cand, take = length - window, budget - window
@@ -106,7 +108,7 @@ def _select_ties_high(scores, length, budget, window):
     return np.asarray(sorted(sorted(range(cand), key=key)[:take]) + list(range(cand, length)))
 
 
-def _select_window_outside(scores, length, budget, window):
+def _select_window_outside(scores, length, budget, window, sinks=0):
     if length <= budget:
         return np.arange(length)
     cand = length - window
@@ -115,12 +117,35 @@ def _select_window_outside(scores, length, budget, window):
     return np.asarray(sorted(best) + list(range(cand, length)))
 
 
-def _select_nan_high(scores, length, budget, window):
+def _select_nan_high(scores, length, budget, window, sinks=0):
     if length <= budget:
         return np.arange(length)
     cand, take = length - window, budget - window
     key = lambda t: (-(math.inf if math.isnan(scores[t]) else scores[t]), t)  # noqa: E731
     return np.asarray(sorted(sorted(range(cand), key=key)[:take]) + list(range(cand, length)))
+
+
+def _select_sinks_outside(scores, length, budget, window, sinks=0):
+    # sinks added on top of the budget instead of inside it
+    if length <= budget:
+        return np.arange(length)
+    cand, take = length - window, budget - window
+    key = lambda t: (-(-math.inf if math.isnan(scores[t]) else scores[t]), t)  # noqa: E731
+    best = sorted(range(sinks, cand), key=key)[:take]
+    return np.asarray(list(range(sinks)) + sorted(best) + list(range(cand, length)))
+
+
+def _unit_scores_max_is_mean(keys, qbar, qabs, R, p, deltas, base, aggregate="mean"):
+    G = qbar.shape[0]
+    return sum(T.head_score(keys, qbar[g], qabs[g], R[g], p, deltas, base) for g in range(G)) / G
+
+
+_compress_step = T.compress_step
+
+
+def _compress_step_trigger_ignored(*args, **kw):
+    kw["trigger"] = 0
+    return _compress_step(*args, **kw)
 
 
 def _compact_off_by_one(rows, idx):
@@ -164,6 +189,9 @@ MUTATIONS = [
     ("select", _select_ties_high),
     ("select", _select_window_outside),
     ("select", _select_nan_high),
+    ("select", _select_sinks_outside),
+    ("unit_scores", _unit_scores_max_is_mean),
+    ("compress_step", _compress_step_trigger_ignored),
     ("compact_rows", _compact_off_by_one),
     ("freed_blocks", _freed_floor),
     ("calibrate", _calibrate_vector_norms),

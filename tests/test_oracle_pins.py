@@ -467,3 +467,87 @@ def test_page_memory_ratios():
         assert round(T / len(idx), c["reduction_decimals"]) == c["reduction_printed"]
         freed = oracle.freed_blocks(list(range(T // 16)), T, len(idx), 16)
         assert len(freed) == (T - B) // 16
+
+
+# ---------------------------------------------------------------------------
+# Variants: attention sinks, compression trigger, max over the GQA group
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("seed", range(20))
+def test_select_with_sinks_brute_force(seed):
+    """With s sinks: slots [0, s) and the last W slots are kept, plus the
+    best (B - W - s) of the slots between, by (score desc, slot asc)."""
+    rng = np.random.default_rng(300 + seed)
+    length = int(rng.integers(1, 14))
+    budget = int(rng.integers(1, 10))
+    window = int(rng.integers(0, budget + 1))
+    sinks = int(rng.integers(0, budget - window + 1))
+    s = rng.integers(-3, 4, size=length).astype(np.float64)
+    idx = oracle.select(s, length, budget, window, sinks)
+    if length <= budget:
+        assert list(idx) == list(range(length))
+        return
+    cand, take = length - window, budget - window - sinks
+    kept = set(int(i) for i in idx)
+    assert len(kept) == budget and list(idx) == sorted(kept)
+    assert set(range(sinks)) <= kept and set(range(cand, length)) <= kept
+    chosen = kept - set(range(sinks)) - set(range(cand, length))
+    pool = range(sinks, cand)
+    winners = [set(c) for c in itertools.combinations(pool, take)
+               if all(_dominates(s, a, b) for a in c for b in pool if b not in c)]
+    assert winners == [chosen]
+
+
+def test_select_sinks_special_cases():
+    inc = np.arange(20, dtype=np.float64)                 # later slots score higher
+    assert list(oracle.select(inc, 20, 8, 3, 2)) == [0, 1, 14, 15, 16, 17, 18, 19]
+    assert list(oracle.select(inc, 20, 8, 3, 0)) == [12, 13, 14, 15, 16, 17, 18, 19]
+    assert list(oracle.select(inc, 20, 8, 0, 8)) == list(range(8))
+    with pytest.raises(ValueError):
+        oracle.select(inc, 20, 8, 5, 4)
+
+
+def test_trigger_leaves_short_sequences_alone():
+    rng = np.random.default_rng(19)
+    L, Hkv, G, D, bs = 1, 1, 1, 8, 4
+    k = rng.normal(size=(L, 12, Hkv, bs, D))
+    kb = np.arange(k.size, dtype=np.int64).reshape(k.shape)
+    table = np.arange(12).reshape(3, 4)
+    qbar = rng.normal(size=(L, 1, D))
+    qabs = np.abs(oracle.as_bands(qbar)) + 0.2
+    R = np.array([[0.5]])
+    lens = [10, 14, 16]
+    out = oracle.compress_step(k, kb, -kb, table, lens, [20, 20, 20], qbar, qabs, R, G, [1], 1e4,
+                               budget=8, window=2, trigger=12)
+    assert out["seq_len"] == [10, 8, 8]                  # 10 <= trigger untouched
+    np.testing.assert_array_equal(out["k_pool"][0, 0:3], kb[0, 0:3])
+    assert out["freed_ids"] == [int(table[1, 2]), int(table[1, 3]), int(table[2, 2]), int(table[2, 3])]
+    low = oracle.compress_step(k, kb, -kb, table, lens, [20, 20, 20], qbar, qabs, R, G, [1], 1e4,
+                               budget=8, window=2, trigger=3)   # below the budget: the budget
+    assert low["seq_len"] == [8, 8, 8]
+
+
+def test_max_over_group_matches_per_head_brute_force():
+    """aggregate='max' is the largest of the G per-head scores, each from the
+    mean rotated-centre logit (explicit rotation matrices) plus its norm term."""
+    rng = np.random.default_rng(20)
+    D, G, base, p = 8, 3, 1e4, 50
+    deltas = [1, 3, 9]
+    T = 12
+    pos = rng.integers(0, p, size=T)
+    k_pre = rng.normal(size=(T, D))
+    k_post = np.stack([_rotate_explicit(k_pre[t], pos[t], base) for t in range(T)])
+    qbar = rng.normal(size=(G, D))
+    qmag = np.abs(oracle.as_bands(qbar))
+    A = qmag + rng.uniform(0.1, 1.0, size=(G, D // 2))
+    R = rng.uniform(0.2, 0.9, size=G)
+    per_head = np.zeros((G, T))
+    for g in range(G):
+        for t in range(T):
+            trig = np.mean([_rotate_explicit(qbar[g], p + d, base) @ k_post[t] for d in deltas])
+            bands = np.hypot(k_pre[t, :D // 2], k_pre[t, D // 2:])
+            per_head[g, t] = trig + (1 - R[g]) * float(((A[g] - qmag[g]) * bands).sum())
+    got = oracle.unit_scores(k_post, qbar, A, R, p, deltas, base, aggregate="max")
+    np.testing.assert_allclose(got, per_head.max(axis=0), rtol=1e-10, atol=1e-12)
+    one = oracle.unit_scores(k_post, qbar[:1], A[:1], R[:1], p, deltas, base, aggregate="max")
+    np.testing.assert_allclose(one, oracle.unit_scores(k_post, qbar[:1], A[:1], R[:1], p, deltas, base), rtol=1e-14)
