@@ -56,6 +56,10 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target oracle sample time")
+    ap.add_argument("--sinks", type=int, default=0, help="leading slots always kept (variant)")
+    ap.add_argument("--trigger", type=int, default=0, help="compress only sequences longer than this (variant)")
+    ap.add_argument("--aggregate", choices=["mean", "max"], default="mean",
+                    help="GQA aggregation of the per-head scores (variant)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling cases of the same kernels)")
     return ap.parse_args()
@@ -192,7 +196,7 @@ def unit_rows(pool, table_row, length, l, h):
 
 # ---------------------------------------------------------- oracle sample
 
-def oracle_sample(units, stats_fn, deltas, base, budget, window, seconds):
+def oracle_sample(units, stats_fn, deltas, base, budget, window, seconds, sinks=0, aggregate="mean"):
     """Time the float64 oracle on units until about ``seconds`` have passed.
 
     ``units`` yields (keys_bf16_cpu [T,128], vals_bf16_cpu, (s, l, h), p).
@@ -212,7 +216,7 @@ def oracle_sample(units, stats_fn, deltas, base, budget, window, seconds):
         kf = keys.double().numpy()
         kb, vb = keys.view(torch.int16).numpy(), vals.view(torch.int16).numpy()
         t0 = time.perf_counter()
-        oracle.compress_unit(kf, kb, vb, qb, qa, r, p, deltas, base, budget, window)
+        oracle.compress_unit(kf, kb, vb, qb, qa, r, p, deltas, base, budget, window, sinks, aggregate)
         t_used += time.perf_counter() - t0
         keys_done += kf.shape[0]
         n += 1
@@ -258,10 +262,14 @@ def run_ours(args, world, rank, local, dist):
 
     lens = wl.seq_len.cpu().tolist()
     kept_blocks = [min((n + 15) // 16, (B + 15) // 16) for n in lens]
-    keys_per_step = sum(lens) * L * Hkv
+    trig = max(args.trigger, B)
+    keys_per_step = sum(n for n in lens if n > trig) * L * Hkv      # keys of the sequences the step compresses
     cache = tri.KvCache(wl.k_pool, wl.v_pool, wl.block_table, wl.seq_len, wl.cur_pos,
                         torch.zeros(1, dtype=torch.int32, device=dev), G)
-    ws = tri.alloc_workspace(cache, B)
+    variant = (args.sinks, args.trigger, args.aggregate) != (0, 0, "mean")
+    opt = tri.step_options(B, W, args.sinks, args.trigger,
+                           tri.TRI_AGG_MAX if args.aggregate == "max" else tri.TRI_AGG_MEAN)
+    ws = tri.alloc_workspace(cache, opt)
     freed = torch.empty(S * wl.max_blocks, dtype=torch.int32, device=dev)
     count = torch.empty(1, dtype=torch.int32, device=dev)
 
@@ -279,8 +287,12 @@ def run_ours(args, world, rank, local, dist):
         flush.zero_()
 
     def step(events=None, idx_out=None):
-        tri.tri_compress_step(cache, qbar, qabs, R, cfg.base, wl.deltas, B, W, freed, count, ws,
-                              idx_out=idx_out, events=events)
+        if variant:
+            tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, freed_ids=freed,
+                                     freed_count=count, idx_out=idx_out, events=events)
+        else:
+            tri.tri_compress_step(cache, qbar, qabs, R, cfg.base, wl.deltas, B, W, freed, count, ws,
+                                  idx_out=idx_out, events=events)
 
     # census (untimed): how many rows a step moves, from its kept indices
     idx = torch.empty(S, L, Hkv, B, dtype=torch.int32, device=dev)
@@ -290,7 +302,7 @@ def run_ours(args, world, rank, local, dist):
         raise RuntimeError("device status flag raised by the census step")
     moved = 0
     for s in range(S):
-        if lens[s] > B:
+        if lens[s] > trig:
             j = torch.arange(B, device=dev, dtype=torch.int32)
             moved += int((idx[s] != j).sum().item())
     del idx
@@ -363,8 +375,8 @@ def run_ours(args, world, rank, local, dist):
     # ------------------------------------------------------------ e2e
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, tri, cache, wl, cfg, qbar, qabs, R, ws, freed, count, save_k, save_v, rblocks,
-                      save_len, keys_per_step, dev, world, dist)
+        e2e = run_e2e(args, tri, cache, wl, qbar, qabs, R, freed, count, save_k, save_v, rblocks,
+                      save_len, keys_per_step, dev, world, dist, step)
 
     # ---------------------------------------------------- cpu baseline
     cpu = None
@@ -378,6 +390,7 @@ def run_ours(args, world, rank, local, dist):
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "seq_lens": lens,
                    "budget": B, "window": W, "rope_base": cfg.base, "deltas": wl.deltas,
+                   "sinks": args.sinks, "trigger": trig, "aggregate": args.aggregate,
                    "keys_per_step_per_gpu": keys_per_step, "freed_blocks_per_step": job_freed,
                    "parallelism": f"units sharded: one independent cache per GPU x{world}",
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
@@ -391,8 +404,8 @@ def run_ours(args, world, rank, local, dist):
         print(json.dumps(out), flush=True)
 
 
-def run_e2e(args, tri, cache, wl, cfg, qbar, qabs, R, ws, freed, count, save_k, save_v, rblocks, save_len,
-            keys_per_step, dev, world, dist):
+def run_e2e(args, tri, cache, wl, qbar, qabs, R, freed, count, save_k, save_v, rblocks, save_len,
+            keys_per_step, dev, world, dist, step):
     """Same step through the C ABI with the cache in pinned HOST memory: the
     timed region copies the inputs in, runs the step, and copies the result
     (the kept region of K/V, new lengths, freed ids and count) back."""
@@ -419,7 +432,7 @@ def run_e2e(args, tri, cache, wl, cfg, qbar, qabs, R, ws, freed, count, save_k, 
         a.record()
         for n, t in host.items():
             dev_in[n].copy_(t, non_blocking=True)
-        tri.tri_compress_step(cache, qbar, qabs, R, cfg.base, wl.deltas, cfg.budget, cfg.window, freed, count, ws)
+        step()
         out_k.copy_(wl.k_pool[:, rblocks], non_blocking=True)
         out_v.copy_(wl.v_pool[:, rblocks], non_blocking=True)
         out_len.copy_(wl.seq_len, non_blocking=True)
@@ -471,7 +484,7 @@ def run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens):
                    (s, l, h), int(wl.cur_pos[s].item()))
 
     keys, secs, n = oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
-                                  args.cpu_seconds)
+                                  args.cpu_seconds, args.sinks, args.aggregate)
     return {"value": round(keys / secs, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
             "sample": f"{n} random units of this workload ({keys} keys), float64 numpy oracle, 1 thread; "
                       f"host has {os.cpu_count()} cores", "seconds": round(secs, 2)}
@@ -518,11 +531,12 @@ def run_reference(args, world, rank):
 
     it = units()
     for _ in range(args.warmup):
-        oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, 0.0)
+        oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, 0.0, args.sinks, args.aggregate)
     keys = secs = 0.0
     n_units = 0
     for _ in range(args.steps):
-        k, s_, n = oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, per_step)
+        k, s_, n = oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, per_step,
+                                 args.sinks, args.aggregate)
         keys += k
         secs += s_
         n_units += n

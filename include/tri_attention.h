@@ -209,7 +209,8 @@ tri_status tri_select_topk(const tri_kv_desc *desc, const float *scores, int bud
  * freed_ids (sequence order, table order); *freed_count = their number.
  *   idx   : int32 [S][L][Hkv][budget], each unit's first kept[s] entries
  *           strictly ascending and < seq_len[s] (as from tri_select_topk)
- *   kept  : int32 [S], 0 <= kept[s] <= seq_len[s]
+ *   kept  : int32 [S], 0 <= kept[s] <= seq_len[s], and kept[s] <= budget
+ *           unless kept[s] == seq_len[s] (the sequence is left as it is)
  *   freed_ids   : int32 [S*max_blocks] out;  freed_count : int32 [1] out
  * The block table is not modified; the caller truncates it.
  * Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED, TRI_ERR_CUDA.  Device flags:
@@ -273,10 +274,145 @@ tri_status tri_compress_step_static_scratch(tri_kv_desc *desc, const float *qbar
                                             int n_deltas, int budget, int window, int32_t *freed_ids,
                                             int32_t *freed_count, int32_t *idx_out, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Variants of the step.
+ *
+ * tri_step_options gathers the knobs of the selection and of the GQA
+ * aggregation; the plain entry points above are the defaults
+ * {budget, window, 0, 0, TRI_AGG_MEAN}.
+ *
+ *   budget    : B, slots kept per unit, 1 <= B <= TRI_MAX_BUDGET.
+ *   window    : W, the last W slots are always kept (inside B).
+ *   sinks     : the first `sinks` slots (the oldest tokens of the sequence)
+ *               are always kept, also inside B: sinks + W <= B.  With
+ *               sinks > 0 the selection ranks only slots [sinks, len - W)
+ *               and keeps the best B - W - sinks of them.  ([Digest] "Key
+ *               Concepts" and [GeoTrick] "The Core Idea" note that attention
+ *               mass concentrates on a few early positions; keeping them is
+ *               an option of this library, not a step of the method.)
+ *   trigger   : a sequence is compressed only when seq_len > max(trigger, B);
+ *               shorter sequences are left untouched.  0 means B.  A caller
+ *               that appends chunks of C tokens between steps and sets
+ *               trigger = B + C compresses once per chunk instead of after
+ *               every token ([GeoTrick] "Why Existing KV Cache Compression
+ *               Breaks in Production": eviction in whole chunks).
+ *   aggregate : how the G query heads of a KV head combine into one key
+ *               score.  TRI_AGG_MEAN: their mean, folded into one effective
+ *               query (what tri_build_query computes).  TRI_AGG_MAX: their
+ *               maximum, each head scored on its own; G must be 1, 2, 4 or 8
+ *               (TRI_ERR_UNSUPPORTED otherwise).
+ * ---------------------------------------------------------------------- */
+#define TRI_AGG_MEAN 0
+#define TRI_AGG_MAX  1
+
+typedef struct {
+    int budget;
+    int window;
+    int sinks;
+    int trigger;
+    int aggregate;
+} tri_step_options;
+
+/*
+ * A device-resident stack of free paged-block ids, so that a decode loop can
+ * compress and grow its sequences without the host reading freed ids back.
+ *   ids      : int32 [capacity]; entries [0, *count) are free block ids
+ *   count    : int32 [1], device; the number of valid entries
+ *   capacity : entries ids can hold
+ * The library pushes freed blocks on top (tri_compress_step_ex) and pops
+ * from the top (tri_reserve_blocks).  Only the calls it is passed to touch it.
+ */
+typedef struct {
+    int32_t *ids;
+    int32_t *count;
+    int capacity;
+} tri_free_list;
+
+/* Device status bit: a free list had too few entries (pop) or too little
+ * room (push); that call changed neither the list nor the block table. */
+#define TRI_DEVFLAG_FREELIST   8
+#define TRI_ERR_FREELIST       8  /* tri_sync_status: TRI_DEVFLAG_FREELIST */
+
+/* Workspace bytes of tri_score_ex / tri_compress_step_ex with these options
+ * (TRI_AGG_MAX keeps G coefficient sets per unit).  0 if invalid. */
+size_t tri_workspace_size_ex(const tri_kv_desc *desc, const tri_step_options *opt);
+
+/*
+ * tri_score_ex - tri_score with a choice of aggregation.  TRI_AGG_MEAN is
+ * tri_score.  TRI_AGG_MAX writes, for every key,
+ *   max_g [ sum_i Re(qbar_{g,i} m_i conj(K band i))
+ *           + (1 - R_g)(qabs_{g,i} - |qbar_{g,i}|)|K band i| ].
+ *   workspace : >= tri_workspace_size_ex(desc, {1, 0, 0, 0, aggregate}).
+ * Errors and flags: as tri_score; TRI_ERR_UNSUPPORTED for TRI_AGG_MAX with
+ * G not in {1, 2, 4, 8}; TRI_ERR_INVALID for an unknown aggregate.
+ */
+tri_status tri_score_ex(const tri_kv_desc *desc, const float *qbar, const float *qabs,
+                        const float *R, double rope_base, const int32_t *deltas, int n_deltas,
+                        int aggregate, float *scores, void *workspace, size_t ws_bytes,
+                        cudaStream_t stream);
+
+/*
+ * tri_select_topk_ex - tri_select_topk with sinks and a trigger: a unit of
+ * len <= max(trigger, budget) keeps every slot (kept = len; when len > B the
+ * idx entries are 0 .. B-1, as there is room for no more); otherwise it
+ * keeps slots [0, sinks), the last W slots and the best B - W - sinks of the
+ * slots between (score descending, slot ascending), kept = B.  tri_compact_kv
+ * leaves a sequence with kept == seq_len untouched, so the two chain.
+ * opt->aggregate is ignored.  Errors: as tri_select_topk, and
+ * TRI_ERR_INVALID for sinks < 0, sinks + W > B or trigger < 0.
+ */
+tri_status tri_select_topk_ex(const tri_kv_desc *desc, const float *scores,
+                              const tri_step_options *opt, int32_t *idx, int32_t *kept,
+                              cudaStream_t stream);
+
+/*
+ * tri_compress_step_ex - tri_compress_step with options and an optional
+ * device free list.
+ *   opt        : the options above (not NULL).
+ *   free_list  : NULL, or a free list that receives the freed block ids: they
+ *                are pushed on top in the order tri_compress_step reports
+ *                them, and *free_list->count grows by their number.  If the
+ *                list lacks room, nothing is pushed and TRI_DEVFLAG_FREELIST
+ *                is raised (the cache is still compacted and freed_ids, when
+ *                given, still lists the blocks).
+ *   freed_ids, freed_count : as tri_compress_step; may both be NULL when a
+ *                free list is given.
+ *   workspace  : >= tri_workspace_size_ex(desc, opt) bytes.
+ * Sequences with seq_len <= max(trigger, budget) are left untouched.
+ * Errors and flags: as tri_compress_step, plus TRI_DEVFLAG_FREELIST.
+ */
+tri_status tri_compress_step_ex(tri_kv_desc *desc, const float *qbar, const float *qabs,
+                                const float *R, double rope_base, const int32_t *deltas,
+                                int n_deltas, const tri_step_options *opt,
+                                const tri_free_list *free_list, int32_t *freed_ids,
+                                int32_t *freed_count, int32_t *idx_out, void *workspace,
+                                size_t ws_bytes, const tri_phase_events *events,
+                                cudaStream_t stream);
+
+/*
+ * tri_reserve_blocks - grow sequences by n_new[s] slots each, taking the
+ * paged blocks they newly need from the top of a device free list
+ * ([GeoTrick] "Why Existing KV Cache Compression Breaks in Production": the
+ * paged allocator hands out whole blocks).
+ *   block_table : int32 [S][max_blocks], the descriptor's table, writable;
+ *                 entries ceil(seq_len/16) .. ceil((seq_len+n_new)/16) - 1 of
+ *                 sequence s are set.  Sequences take the popped ids in
+ *                 sequence order, each sequence in table order, from the
+ *                 lowest of the popped entries up.
+ *   n_new       : int32 [S], device, >= 0.
+ * seq_len is NOT changed: the caller writes the new rows and then raises it.
+ * All or nothing: if the list holds fewer ids than needed, or a sequence
+ * would exceed max_blocks*16 slots, nothing changes and the device flags
+ * FREELIST or BOUNDS are raised.
+ * Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED, TRI_ERR_CUDA.
+ */
+tri_status tri_reserve_blocks(const tri_kv_desc *desc, int32_t *block_table, const int32_t *n_new,
+                              const tri_free_list *free_list, cudaStream_t stream);
+
 /*
  * tri_sync_status - wait for `stream`, read the device status word, clear it,
  * and return TRI_OK or the error its bits name (BOUNDS before TIMEOUT before
- * NONFINITE).  TRI_ERR_CUDA if the stream itself reports an error.
+ * FREELIST before NONFINITE).  TRI_ERR_CUDA if the stream itself reports an error.
  */
 tri_status tri_sync_status(int32_t *status, cudaStream_t stream);
 

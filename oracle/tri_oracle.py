@@ -251,7 +251,8 @@ def store_unit_rows(pool: np.ndarray, table_row: Sequence[int], rows: np.ndarray
 
 def compress_unit(keys_f64: np.ndarray, k_rows: np.ndarray, v_rows: np.ndarray,
                   qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray, p: int,
-                  deltas: Sequence[int], base: float, budget: int, window: int):
+                  deltas: Sequence[int], base: float, budget: int, window: int,
+                  sinks: int = 0, aggregate: str = "mean"):
     """Score, select and compact one unit.
 
     ``keys_f64`` are the unit's keys widened to float64; ``k_rows`` /
@@ -260,8 +261,8 @@ def compress_unit(keys_f64: np.ndarray, k_rows: np.ndarray, v_rows: np.ndarray,
     new_k_rows, new_v_rows).
     """
     length = keys_f64.shape[0]
-    s = unit_scores(keys_f64, qbar, qabs, R, p, deltas, base)
-    idx = select(s, length, budget, window)
+    s = unit_scores(keys_f64, qbar, qabs, R, p, deltas, base, aggregate)
+    idx = select(s, length, budget, window, sinks)
     return s, idx, compact_rows(k_rows, idx), compact_rows(v_rows, idx)
 
 

@@ -28,6 +28,10 @@ TRI_ERR_DEVICE_BOUNDS = 4
 TRI_ERR_TIMEOUT = 5
 TRI_ERR_NONFINITE = 6
 TRI_ERR_WORKSPACE = 7
+TRI_ERR_FREELIST = 8
+
+TRI_AGG_MEAN = 0
+TRI_AGG_MAX = 1
 
 TRI_HEAD_DIM = 128
 TRI_BLOCK_SIZE = 16
@@ -38,7 +42,8 @@ TRI_MAX_BUDGET = 16384
 EXPORTS = (
     "tri_calibrate_centers", "tri_build_query", "tri_workspace_size", "tri_score",
     "tri_select_topk", "tri_compact_kv", "tri_compress_step", "tri_compress_step_static_scratch",
-    "tri_sync_status", "tri_status_string",
+    "tri_sync_status", "tri_status_string", "tri_workspace_size_ex", "tri_score_ex", "tri_select_topk_ex",
+    "tri_compress_step_ex", "tri_reserve_blocks",
 )
 TRI_STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -70,6 +75,53 @@ class TriPhaseEvents(ctypes.Structure):
                 ("after_score", ctypes.c_void_p), ("after_evict", ctypes.c_void_p)]
 
 
+class TriStepOptions(ctypes.Structure):
+    """Mirror of ``tri_step_options``."""
+
+    _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
+                ("trigger", ctypes.c_int), ("aggregate", ctypes.c_int)]
+
+
+class TriFreeList(ctypes.Structure):
+    """Mirror of ``tri_free_list``."""
+
+    _fields_ = [("ids", ctypes.c_void_p), ("count", ctypes.c_void_p), ("capacity", ctypes.c_int)]
+
+
+class FreeList:
+    """A device-resident stack of free block ids (int32 ``ids`` of length
+    capacity, int32 ``count`` of one element), kept alive with its mirror."""
+
+    def __init__(self, ids: torch.Tensor, count: torch.Tensor):
+        if ids.dim() != 1 or count.numel() != 1:
+            raise ValueError("ids must be 1-D and count a single element")
+        self.ids, self.count = ids, count
+        self.c = TriFreeList(ids=_ptr(ids, torch.int32, "ids"), count=_ptr(count, torch.int32, "count"),
+                             capacity=ids.numel())
+
+    @classmethod
+    def from_ids(cls, free_ids, capacity: int, device) -> "FreeList":
+        ids = torch.full((capacity,), -1, dtype=torch.int32, device=device)
+        free = torch.as_tensor(list(free_ids), dtype=torch.int32)
+        if free.numel() > capacity:
+            raise ValueError("more free ids than capacity")
+        ids[:free.numel()] = free.to(device)
+        return cls(ids, torch.tensor([free.numel()], dtype=torch.int32, device=device))
+
+    def contents(self):
+        n = int(self.count.item())
+        return [int(x) for x in self.ids[:n].tolist()]
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def step_options(budget: int, window: int, sinks: int = 0, trigger: int = 0,
+                 aggregate: int = TRI_AGG_MEAN) -> TriStepOptions:
+    return TriStepOptions(int(budget), int(window), int(sinks), int(trigger), int(aggregate))
+
+
 _lib: Optional[ctypes.CDLL] = None
 
 
@@ -92,6 +144,13 @@ def _load() -> ctypes.CDLL:
                                   ctypes.POINTER(TriPhaseEvents), P]),
         "tri_compress_step_static_scratch": (I, [desc_p, P, P, P, D, P, I, I, I, P, P, P, P]),
         "tri_sync_status": (I, [P, P]),
+        "tri_workspace_size_ex": (S, [desc_p, ctypes.POINTER(TriStepOptions)]),
+        "tri_score_ex": (I, [desc_p, P, P, P, D, P, I, I, P, P, S, P]),
+        "tri_select_topk_ex": (I, [desc_p, P, ctypes.POINTER(TriStepOptions), P, P, P]),
+        "tri_compress_step_ex": (I, [desc_p, P, P, P, D, P, I, ctypes.POINTER(TriStepOptions),
+                                     ctypes.POINTER(TriFreeList), P, P, P, P, S,
+                                     ctypes.POINTER(TriPhaseEvents), P]),
+        "tri_reserve_blocks": (I, [desc_p, P, P, ctypes.POINTER(TriFreeList), P]),
         "tri_status_string": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -223,22 +282,26 @@ def tri_compact_kv(cache: KvCache, idx, kept, budget: int, freed_ids, freed_coun
     _check(code, "tri_compact_kv")
 
 
+def _events(events):
+    if events is None:
+        return None
+    handles = []
+    for e in events:
+        if e is None:
+            handles.append(None)
+            continue
+        if e.cuda_event == 0:          # torch creates the CUDA event lazily
+            e.record()
+        handles.append(ctypes.c_void_p(e.cuda_event))
+    return ctypes.byref(TriPhaseEvents(*handles))
+
+
 def tri_compress_step(cache: KvCache, qbar, qabs, R, rope_base: float, deltas, budget: int, window: int,
                       freed_ids, freed_count, workspace, idx_out=None, events=None, stream=None) -> None:
     """``events``: optional sequence of four recorded-or-fresh torch.cuda.Event
     (start, after_query, after_score, after_evict), each with enable_timing."""
     arr, n = _deltas(deltas)
-    ev = None
-    if events is not None:
-        handles = []
-        for e in events:
-            if e is None:
-                handles.append(None)
-                continue
-            if e.cuda_event == 0:          # torch creates the CUDA event lazily
-                e.record()
-            handles.append(ctypes.c_void_p(e.cuda_event))
-        ev = ctypes.byref(TriPhaseEvents(*handles))
+    ev = _events(events)
     code = library().tri_compress_step(
         cache.ref, _ptr(qbar, torch.float32, "qbar"), _ptr(qabs, torch.float32, "qabs"),
         _ptr(R, torch.float32, "R"), float(rope_base), arr, n, int(budget), int(window),
@@ -263,15 +326,65 @@ def tri_compress_step_static_scratch(cache: KvCache, qbar, qabs, R, rope_base: f
     _check(code, "tri_compress_step_static_scratch")
 
 
+def tri_workspace_size_ex(cache: KvCache, opt: TriStepOptions) -> int:
+    return int(library().tri_workspace_size_ex(cache.ref, ctypes.byref(opt)))
+
+
+def tri_score_ex(cache: KvCache, qbar, qabs, R, rope_base: float, deltas, aggregate: int, scores, workspace,
+                 stream=None) -> None:
+    arr, n = _deltas(deltas)
+    code = library().tri_score_ex(
+        cache.ref, _ptr(qbar, torch.float32, "qbar"), _ptr(qabs, torch.float32, "qabs"),
+        _ptr(R, torch.float32, "R"), float(rope_base), arr, n, int(aggregate),
+        _ptr(scores, torch.float32, "scores"), _ptr(workspace, torch.uint8, "workspace"), workspace.numel(),
+        _stream(stream))
+    _check(code, "tri_score_ex")
+
+
+def tri_select_topk_ex(cache: KvCache, scores, opt: TriStepOptions, idx, kept, stream=None) -> None:
+    code = library().tri_select_topk_ex(
+        cache.ref, _ptr(scores, torch.float32, "scores"), ctypes.byref(opt), _ptr(idx, torch.int32, "idx"),
+        _ptr(kept, torch.int32, "kept"), _stream(stream))
+    _check(code, "tri_select_topk_ex")
+
+
+def tri_compress_step_ex(cache: KvCache, qbar, qabs, R, rope_base: float, deltas, opt: TriStepOptions,
+                         workspace, free_list: Optional[FreeList] = None, freed_ids=None, freed_count=None,
+                         idx_out=None, events=None, stream=None) -> None:
+    arr, n = _deltas(deltas)
+    code = library().tri_compress_step_ex(
+        cache.ref, _ptr(qbar, torch.float32, "qbar"), _ptr(qabs, torch.float32, "qabs"),
+        _ptr(R, torch.float32, "R"), float(rope_base), arr, n, ctypes.byref(opt),
+        free_list.ref if free_list is not None else None,
+        _ptr(freed_ids, torch.int32, "freed_ids", allow_none=True),
+        _ptr(freed_count, torch.int32, "freed_count", allow_none=True),
+        _ptr(idx_out, torch.int32, "idx_out", allow_none=True),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _events(events), _stream(stream))
+    _check(code, "tri_compress_step_ex")
+
+
+def tri_reserve_blocks(cache: KvCache, n_new, free_list: FreeList, stream=None) -> None:
+    """Pop the blocks that n_new[s] more slots per sequence need from the
+    free list into the cache's block table (seq_len is not changed)."""
+    code = library().tri_reserve_blocks(
+        cache.ref, _ptr(cache.tensors[2], torch.int32, "block_table"), _ptr(n_new, torch.int32, "n_new"),
+        free_list.ref, _stream(stream))
+    _check(code, "tri_reserve_blocks")
+
+
 def tri_sync_status(status, stream=None) -> int:
     """Wait for the stream, read and clear the device status word; returns the code."""
     return int(library().tri_sync_status(_ptr(status, torch.int32, "status"), _stream(stream)))
 
 
-def alloc_workspace(cache: KvCache, budget: int, device=None) -> torch.Tensor:
-    """A uint8 workspace of tri_workspace_size bytes (torch allocations are
-    256-byte aligned)."""
-    n = tri_workspace_size(cache, budget)
+def alloc_workspace(cache: KvCache, budget, device=None) -> torch.Tensor:
+    """A uint8 workspace of tri_workspace_size bytes, or of
+    tri_workspace_size_ex bytes when ``budget`` is a TriStepOptions (torch
+    allocations are 256-byte aligned)."""
+    if isinstance(budget, TriStepOptions):
+        n = tri_workspace_size_ex(cache, budget)
+    else:
+        n = tri_workspace_size(cache, budget)
     if n == 0:
         raise TriError(TRI_ERR_INVALID, "tri_workspace_size")
     ws = torch.empty(n, dtype=torch.uint8, device=device or cache.tensors[0].device)

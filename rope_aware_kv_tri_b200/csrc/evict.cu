@@ -156,9 +156,9 @@ __device__ void pick_digit(const int* hist, int nb, int shift, uint32_t& prefix,
     mask |= (uint32_t)(nb - 1) << shift;
 }
 
-// Pass 1: histogram of the top key bits of all candidates.  Returns whether
-// a NaN score was seen.
-__device__ bool top_histogram(const float* __restrict__ sc, int cand, int* hist) {
+// Pass 1: histogram of the top key bits of candidates [lo, cand).  Returns
+// whether a NaN score was seen.
+__device__ bool top_histogram(const float* __restrict__ sc, int cand, int lo, int* hist) {
     for (int i = threadIdx.x; i < kTopBins; i += kEvictThreads) hist[i] = 0;
     __syncthreads();
     bool nan_seen = false;
@@ -177,13 +177,15 @@ __device__ bool top_histogram(const float* __restrict__ sc, int cand, int* hist)
                 const float e[4] = {x[k].x, x[k].y, x[k].z, x[k].w};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    nan_seen |= isnan(e[c]);
-                    atomicAdd(&hist[order_key(e[c]) >> kTopShift], 1);
+                    if (4 * (v0 + k * kEvictThreads) + c >= lo) {
+                        nan_seen |= isnan(e[c]);
+                        atomicAdd(&hist[order_key(e[c]) >> kTopShift], 1);
+                    }
                 }
             }
         }
     }
-    for (int t = 4 * nvec + threadIdx.x; t < cand; t += kEvictThreads) {
+    for (int t = max(4 * nvec, lo) + threadIdx.x; t < cand; t += kEvictThreads) {
         const float e = sc[t];
         nan_seen |= isnan(e);
         atomicAdd(&hist[order_key(e) >> kTopShift], 1);
@@ -204,13 +206,13 @@ __device__ __forceinline__ void load4(const float* __restrict__ sc, int t, int e
 
 // Streaming radix pass over all candidates (fallback when the cut's bucket
 // does not fit the shared list).
-__device__ void stream_radix_pass(const float* __restrict__ sc, int cand, uint32_t& prefix, uint32_t& mask,
+__device__ void stream_radix_pass(const float* __restrict__ sc, int cand, int lo, uint32_t& prefix, uint32_t& mask,
                                   int& rem, int shift, int bits, int* hist, EvictSmem& sm) {
     const int nb = 1 << bits;
     const uint32_t dmask = (uint32_t)nb - 1u;
     for (int i = threadIdx.x; i < nb; i += kEvictThreads) hist[i] = 0;
     __syncthreads();
-    for (int t = threadIdx.x; t < cand; t += kEvictThreads) {
+    for (int t = lo + threadIdx.x; t < cand; t += kEvictThreads) {
         const uint32_t key = order_key(sc[t]);
         if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & dmask], 1);
     }
@@ -344,8 +346,8 @@ __device__ void finish_from_list(const uint32_t* list_key, const int* list_slot,
 // every candidate's linear bucket in shared memory; the bitmap of buckets
 // above the cut's and the cut bucket's slots then come from shared memory,
 // and only the (few) cut-bucket scores are read again.
-__device__ bool select_one_pass(const float* __restrict__ sc, int cand, int take, float lo, float scale, int* sidx,
-                                EvictSmem& sm) {
+__device__ bool select_one_pass(const float* __restrict__ sc, int cand, int first, int take, float lo, float scale,
+                                int* sidx, EvictSmem& sm) {
     OnePassScratch& o = sm.u.sel.one;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     for (int i = threadIdx.x; i < kLinBins; i += kEvictThreads) o.hist[i] = 0;
@@ -367,17 +369,25 @@ __device__ bool select_one_pass(const float* __restrict__ sc, int cand, int take
                 const int b2 = lin_bucket(x[k].z, lo, scale), b3 = lin_bucket(x[k].w, lo, scale);
                 *reinterpret_cast<uint2*>(&o.code[4 * v]) =
                     make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
-                atomicAdd(&o.hist[b0], 1);
-                atomicAdd(&o.hist[b1], 1);
-                atomicAdd(&o.hist[b2], 1);
-                atomicAdd(&o.hist[b3], 1);
+                if (4 * v >= first) {
+                    atomicAdd(&o.hist[b0], 1);
+                    atomicAdd(&o.hist[b1], 1);
+                    atomicAdd(&o.hist[b2], 1);
+                    atomicAdd(&o.hist[b3], 1);
+                } else {
+                    // the first vector holds excluded leading slots
+                    if (4 * v + 0 >= first) atomicAdd(&o.hist[b0], 1);
+                    if (4 * v + 1 >= first) atomicAdd(&o.hist[b1], 1);
+                    if (4 * v + 2 >= first) atomicAdd(&o.hist[b2], 1);
+                    if (4 * v + 3 >= first) atomicAdd(&o.hist[b3], 1);
+                }
             }
         }
     }
     for (int t = 4 * nvec + threadIdx.x; t < cand; t += kEvictThreads) {
         const int b = lin_bucket(sc[t], lo, scale);
         o.code[t] = (uint16_t)b;
-        atomicAdd(&o.hist[b], 1);
+        if (t >= first) atomicAdd(&o.hist[b], 1);
     }
     __syncthreads();
     int rem = take;
@@ -399,7 +409,7 @@ __device__ bool select_one_pass(const float* __restrict__ sc, int cand, int take
             for (int i = 0; i < 8; ++i) {
                 const int t = 8 * q + i;
                 const int b = (int)((cw[i >> 1] >> (16 * (i & 1))) & 0xffffu);
-                if (t < cand) {
+                if (t < cand && t >= first) {
                     if (b > bstar) m |= 1u << i;
                     else if (b == bstar) {
                         const int pos = atomicAdd(&sm.n_list, 1);
@@ -428,8 +438,8 @@ __device__ bool select_one_pass(const float* __restrict__ sc, int cand, int take
 // from the bitmaps in slot order.  Returns false, with nothing kept, when the
 // range is not finite, the candidates exceed the bitmap, or the cut's
 // bucket exceeds the list.
-__device__ bool select_linear(const float* __restrict__ sc, int cand, int take, uint32_t kmin, uint32_t kmax,
-                              int* sidx, EvictSmem& sm) {
+__device__ bool select_linear(const float* __restrict__ sc, int cand, int first, int take, uint32_t kmin,
+                              uint32_t kmax, int* sidx, EvictSmem& sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const float lo = key_value(kmin), hi = key_value(kmax);
     if (kmin > kmax || !isfinite(lo) || !isfinite(hi) || cand > kBitmapWords * 32) return false;
@@ -437,11 +447,11 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
     if (!isfinite(span)) return false;
     if (span == 0.f) {
         // every score of the unit is equal: the lowest slots win every tie
-        for (int j = threadIdx.x; j < take; j += kEvictThreads) sidx[j] = j;
+        for (int j = threadIdx.x; j < take; j += kEvictThreads) sidx[j] = first + j;
         return true;
     }
     const float scale = (float)(kLinBins - 1) / span;
-    if (cand <= kCodeSlots) return select_one_pass(sc, cand, take, lo, scale, sidx, sm);
+    if (cand <= kCodeSlots) return select_one_pass(sc, cand, first, take, lo, scale, sidx, sm);
     int* hist = sm.u.sel.hist;
     // warp segments of whole 128-slot steps
     const int seg = ((cand + kEvictWarps - 1) / kEvictWarps + kStep - 1) / kStep * kStep;
@@ -463,15 +473,16 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
             }
 #pragma unroll
             for (int k = 0; k < kUnroll; ++k) {
+                const int t = 4 * (v0 + k * kEvictThreads);
                 if (v0 + k * kEvictThreads < nvec) {
-                    atomicAdd(&hist[lin_bucket(x[k].x, lo, scale)], 1);
-                    atomicAdd(&hist[lin_bucket(x[k].y, lo, scale)], 1);
-                    atomicAdd(&hist[lin_bucket(x[k].z, lo, scale)], 1);
-                    atomicAdd(&hist[lin_bucket(x[k].w, lo, scale)], 1);
+                    if (t + 0 >= first) atomicAdd(&hist[lin_bucket(x[k].x, lo, scale)], 1);
+                    if (t + 1 >= first) atomicAdd(&hist[lin_bucket(x[k].y, lo, scale)], 1);
+                    if (t + 2 >= first) atomicAdd(&hist[lin_bucket(x[k].z, lo, scale)], 1);
+                    if (t + 3 >= first) atomicAdd(&hist[lin_bucket(x[k].w, lo, scale)], 1);
                 }
             }
         }
-        for (int t = 4 * nvec + threadIdx.x; t < cand; t += kEvictThreads)
+        for (int t = max(4 * nvec, first) + threadIdx.x; t < cand; t += kEvictThreads)
             atomicAdd(&hist[lin_bucket(sc[t], lo, scale)], 1);
     }
     __syncthreads();
@@ -498,7 +509,7 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
                 int n_in = 0;
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const bool valid = t + c < end;
+                    const bool valid = t + c < end && t + c >= first;
                     const int b = lin_bucket(x[k][c], lo, scale);
                     above[c] = __ballot_sync(0xffffffffu, valid && b > bstar);
                     inb[c] = __ballot_sync(0xffffffffu, valid && b == bstar);
@@ -532,8 +543,8 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int take, 
 }
 
 // Smallest and largest order key among the candidates (block reduction).
-__device__ void candidate_key_range(const float* __restrict__ sc, int cand, uint32_t& kmin, uint32_t& kmax,
-                                    EvictSmem& sm) {
+__device__ void candidate_key_range(const float* __restrict__ sc, int cand, int first, uint32_t& kmin,
+                                    uint32_t& kmax, EvictSmem& sm) {
     uint32_t lo = 0xffffffffu, hi = 0u;
     const int nvec = cand >> 2;
     const float4* v4 = reinterpret_cast<const float4*>(sc);
@@ -546,15 +557,19 @@ __device__ void candidate_key_range(const float* __restrict__ sc, int cand, uint
         }
 #pragma unroll
         for (int k = 0; k < kUnroll; ++k) {
+            const int t = 4 * (v0 + k * kEvictThreads);
             if (v0 + k * kEvictThreads < nvec) {
+                // an excluded leading slot takes a neutral key (the range's own bounds)
                 const uint32_t a = order_key(x[k].x), b = order_key(x[k].y);
                 const uint32_t c = order_key(x[k].z), d = order_key(x[k].w);
-                lo = min(lo, min(min(a, b), min(c, d)));
-                hi = max(hi, max(max(a, b), max(c, d)));
+                lo = min(lo, min(min(t + 0 >= first ? a : 0xffffffffu, t + 1 >= first ? b : 0xffffffffu),
+                                 min(t + 2 >= first ? c : 0xffffffffu, t + 3 >= first ? d : 0xffffffffu)));
+                hi = max(hi, max(max(t + 0 >= first ? a : 0u, t + 1 >= first ? b : 0u),
+                                 max(t + 2 >= first ? c : 0u, t + 3 >= first ? d : 0u)));
             }
         }
     }
-    for (int t = 4 * nvec + threadIdx.x; t < cand; t += kEvictThreads) {
+    for (int t = max(4 * nvec, first) + threadIdx.x; t < cand; t += kEvictThreads) {
         const uint32_t k = order_key(sc[t]);
         lo = min(lo, k);
         hi = max(hi, k);
@@ -576,18 +591,28 @@ __device__ void candidate_key_range(const float* __restrict__ sc, int cand, uint
     __syncthreads();
 }
 
+// Kept slots of a unit of len > budget slots: [0, sinks), the best
+// budget - window - sinks of [sinks, len - window), and the last window.
+// The ranking passes run on a 16-byte aligned view that starts at slot
+// a = sinks rounded down to a multiple of 4; the first (sinks - a) slots of
+// the view are excluded, and the view's slot numbers are shifted back by a.
 // kmin_in: whether (kmin, kmax) already bound the unit's score keys.
-__device__ void select_unit(const float* __restrict__ sc, int len, int budget, int window, int* sidx,
-                            EvictSmem& sm, int32_t* status, bool kmin_in, uint32_t kmin, uint32_t kmax) {
-    const int cand = len - window;
-    const int take = budget - window;
+__device__ void select_unit(const float* __restrict__ sc_unit, int len, int budget, int window, int sinks,
+                            int* sidx_unit, EvictSmem& sm, int32_t* status, bool kmin_in, uint32_t kmin,
+                            uint32_t kmax) {
+    const int a = sinks & ~3;
+    const int first = sinks - a;
+    const float* __restrict__ sc = sc_unit + a;
+    int* sidx = sidx_unit + sinks;
+    const int cand = len - window - a;
+    const int take = budget - window - sinks;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     bool done = take == 0;
     if (!done) {
         // A NaN score has the key of -infinity, so it always leaves the range
         // non-finite and takes the streaming path, which flags it.
-        if (!kmin_in) candidate_key_range(sc, cand, kmin, kmax, sm);
-        done = select_linear(sc, cand, take, kmin, kmax, sidx, sm);
+        if (!kmin_in) candidate_key_range(sc, cand, first, kmin, kmax, sm);
+        done = select_linear(sc, cand, first, take, kmin, kmax, sidx, sm);
     }
     if (!done) {
         int* hist = sm.u.sel.hist;
@@ -596,7 +621,7 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
         const int beg = min(warp * seg, cand);
         const int end = min(beg + seg, cand);
 
-        if (top_histogram(sc, cand, hist) && threadIdx.x == 0) raise_flag(status, TRI_DEVFLAG_NONFINITE);
+        if (top_histogram(sc, cand, first, hist) && threadIdx.x == 0) raise_flag(status, TRI_DEVFLAG_NONFINITE);
         uint32_t prefix = 0, mask = 0;
         int rem = take;
         pick_digit(hist, kTopBins, kTopShift, prefix, mask, rem, sm);
@@ -617,7 +642,7 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
                         const int t = t0 + k * kStep + 4 * lane + c;
-                        if (t < end) {
+                        if (t < end && t >= first) {
                             const uint32_t key = order_key(x[k][c]);
                             const uint32_t d = key >> kTopShift;
                             above += d > top ? 1 : 0;
@@ -651,8 +676,8 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
             }
         } else {
             // Fallback: stream the remaining bits, then count per segment.
-            stream_radix_pass(sc, cand, prefix, mask, rem, 10, 10, hist, sm);
-            stream_radix_pass(sc, cand, prefix, mask, rem, 0, 10, hist, sm);
+            stream_radix_pass(sc, cand, first, prefix, mask, rem, 10, 10, hist, sm);
+            stream_radix_pass(sc, cand, first, prefix, mask, rem, 0, 10, hist, sm);
             int gt = 0, eq = 0;
             for (int t0 = beg; t0 < end; t0 += kStep) {
                 float x[4];
@@ -661,8 +686,9 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
                 for (int c = 0; c < 4; ++c) {
                     const int t = t0 + 4 * lane + c;
                     const uint32_t key = order_key(x[c]);
-                    gt += (t < end && key > prefix) ? 1 : 0;
-                    eq += (t < end && key == prefix) ? 1 : 0;
+                    const bool in = t < end && t >= first;
+                    gt += (in && key > prefix) ? 1 : 0;
+                    eq += (in && key == prefix) ? 1 : 0;
                 }
             }
             gt = __reduce_add_sync(0xffffffffu, gt);
@@ -702,8 +728,9 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     const uint32_t key = order_key(x[k][c]);
-                    g[c] = (t + c < end) && key > thr;
-                    e[c] = (t + c < end) && key == thr;
+                    const bool in = t + c < end && t + c >= first;
+                    g[c] = in && key > thr;
+                    e[c] = in && key == thr;
                 }
                 uint32_t eb[4];
                 int eq_lanes = 0, eq_all = 0;
@@ -740,7 +767,11 @@ __device__ void select_unit(const float* __restrict__ sc, int len, int budget, i
             }
         }
     }
-    for (int j = threadIdx.x; j < window; j += kEvictThreads) sidx[take + j] = cand + j;
+    __syncthreads();
+    if (a > 0)
+        for (int j = threadIdx.x; j < take; j += kEvictThreads) sidx[j] += a;
+    for (int j = threadIdx.x; j < sinks; j += kEvictThreads) sidx_unit[j] = j;
+    for (int j = threadIdx.x; j < window; j += kEvictThreads) sidx[take + j] = a + cand + j;
     __syncthreads();
 }
 
@@ -822,18 +853,20 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
     }
     int kept;
     if (p.do_select) {
-        if (len <= p.budget) {
+        if (len <= p.trigger) {
             // Nothing to evict.  A standalone selection reports every slot.
             if (!p.do_compact) {
                 for (int j = threadIdx.x; j < p.budget; j += kEvictThreads)
                     p.idx_out[(int64_t)u * p.budget + j] = j < len ? j : -1;
+                // kept = len; past the budget (a trigger above it) idx only
+                // has room for the first budget slots
                 if (head0 && threadIdx.x == 0) p.kept_out[s] = len;
             }
             return;
         }
         const float* sc = p.scores + (int64_t)u * p.score_stride;
         const bool have_range = p.unit_kmin != nullptr;
-        select_unit(sc, len, p.budget, p.window, sidx, sm, p.status, have_range,
+        select_unit(sc, len, p.budget, p.window, p.sinks, sidx, sm, p.status, have_range,
                     have_range ? p.unit_kmin[u] : 0u, have_range ? p.unit_kmax[u] : 0u);
         kept = p.budget;
         if (p.idx_out)
@@ -845,6 +878,7 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
         if (p.kept_out && head0 && threadIdx.x == 0) p.kept_out[s] = kept;
     } else {
         kept = p.kept_in[s];
+        if (kept == len) return;     // every slot kept: nothing moves (also past the budget)
         if (kept < 0 || kept > len || kept > p.budget) {
             if (threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
             return;
@@ -908,7 +942,13 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
         const int lo = (kept + kBlockRows - 1) / kBlockRows;
         const int hi = (len + kBlockRows - 1) / kBlockRows;
         const int off = p.freed_off[s];
-        for (int e = threadIdx.x; e < hi - lo; e += kEvictThreads) p.freed_ids[off + e] = bt[lo + e];
+        if (p.freed_ids)
+            for (int e = threadIdx.x; e < hi - lo; e += kEvictThreads) p.freed_ids[off + e] = bt[lo + e];
+        if (p.fl_ids) {
+            const int base = __ldcg(p.fl_base);
+            if (base >= 0)
+                for (int e = threadIdx.x; e < hi - lo; e += kEvictThreads) p.fl_ids[base + off + e] = bt[lo + e];
+        }
         if (threadIdx.x == 0) p.seq_len_out[s] = kept;
     }
 }
@@ -1002,7 +1042,7 @@ __global__ void __launch_bounds__(kMoveThreads, 3) move_kernel(const MoveParams 
         const int len = p.lens[s];
         int kept = -1;
         if (len >= 0 && (int64_t)len <= max_len) {
-            kept = p.kept ? p.kept[s] : (len > p.budget ? p.budget : -1);
+            kept = p.kept ? p.kept[s] : (len > p.trigger ? p.budget : -1);
             if (kept > len || kept > p.budget) kept = -1;
         }
         const uint8_t* sk = nullptr;
@@ -1117,7 +1157,78 @@ __global__ void __launch_bounds__(kFinalizeThreads) finalize_kernel(const Finali
     if (threadIdx.x == 0) *p.freed_count = carry;
 }
 
+// Blocks newly needed by sequence s to grow by n slots (0 if invalid).
+__device__ __forceinline__ int blocks_needed(int len, int n, int64_t max_len, bool& bad) {
+    if (len < 0 || n < 0 || (int64_t)len + n > max_len) {
+        bad = true;
+        return 0;
+    }
+    return (int)(((int64_t)len + n + kBlockRows - 1) / kBlockRows - ((int64_t)len + kBlockRows - 1) / kBlockRows);
+}
+
+// One CTA: pop the blocks all sequences need from the top of the free list
+// (all or nothing) and write them into the block table.
+__global__ void __launch_bounds__(kFinalizeThreads) reserve_kernel(const ReserveParams p) {
+    __shared__ int warp_tmp[kFinalizeThreads / 32];
+    const int64_t max_len = (int64_t)p.max_blocks * kBlockRows;
+    bool bad = false;
+    int total = 0;
+    for (int c0 = 0; c0 < p.S; c0 += kFinalizeThreads) {
+        const int s = c0 + threadIdx.x;
+        const int need = s < p.S ? blocks_needed(p.seq_len[s], p.n_new[s], max_len, bad) : 0;
+        int tot;
+        block_exclusive_scan<kFinalizeThreads>(need, warp_tmp, tot);
+        total += tot;
+    }
+    if (__syncthreads_or(bad)) {
+        if (threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
+        return;
+    }
+    const int have = *p.fl_count;
+    if (have > p.fl_capacity) {
+        if (threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
+        return;
+    }
+    if (have < 0 || total > have) {
+        if (threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_FREELIST);
+        return;
+    }
+    const int base = have - total;
+    bool bad_id = false;
+    for (int e = base + threadIdx.x; e < have; e += kFinalizeThreads) {
+        const int b = p.fl_ids[e];
+        bad_id |= (b < 0 || b >= p.num_blocks);
+    }
+    if (__syncthreads_or(bad_id)) {
+        if (threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
+        return;
+    }
+    int carry = 0;
+    for (int c0 = 0; c0 < p.S; c0 += kFinalizeThreads) {
+        const int s = c0 + threadIdx.x;
+        bool unused = false;
+        int need = 0, lo = 0;
+        if (s < p.S) {
+            const int len = p.seq_len[s];
+            need = blocks_needed(len, p.n_new[s], max_len, unused);
+            lo = (len + kBlockRows - 1) / kBlockRows;
+        }
+        int tot;
+        const int ex = block_exclusive_scan<kFinalizeThreads>(need, warp_tmp, tot);
+        for (int e = 0; e < need; ++e)
+            p.block_table[(int64_t)s * p.max_blocks + lo + e] = p.fl_ids[base + carry + ex + e];
+        carry += tot;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) *p.fl_count = base;
+}
+
 }  // namespace
+
+cudaError_t launch_reserve(const ReserveParams& p, cudaStream_t stream) {
+    reserve_kernel<<<1, kFinalizeThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream, bool pdl) {
     const int U = p.S * p.L * p.Hkv;

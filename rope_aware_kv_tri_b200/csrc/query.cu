@@ -17,9 +17,15 @@
 // the GQA group of the per-head trigonometric + weighted-norm score, because
 // both terms are linear in their coefficients.
 //
+// With the max-over-group aggregation the G heads are not folded: head g of
+// unit u gets its own qbar_g m (real dims) and (1 - R_g)(qabs_g - |qbar_g|)
+// at [u][g], and the score kernel takes the largest of the G head scores.
+//
 // The last CTA of the grid (when planning) validates the sequence lengths,
 // copies them to the workspace, and writes the prefix offsets of the score
-// work items and of the freed-block list.
+// work items and of the freed-block list.  A sequence is compressed when its
+// length exceeds the trigger (at least the budget); when a device free list
+// is given it also reserves the list entries the freed ids will fill.
 #include "tri_device.cuh"
 #include "tri_internal.h"
 
@@ -60,6 +66,23 @@ __device__ void build_unit_queries(const QueryParams& p, int b, int ctas_per_seq
     const int u = s * LH + k;
     const int l = k / p.Hkv, h = k % p.Hkv;
     const int Hq = p.Hkv * p.G;
+    if (p.per_head) {
+        for (int g = 0; g < p.G; ++g) {
+            const int64_t row = (int64_t)l * Hq + (int64_t)h * p.G + g;
+            const double xr = p.qbar[row * kHeadDim + i];
+            const double xi = p.qbar[row * kHeadDim + i + kBands];
+            const int64_t o = (int64_t)u * p.G + g;
+            p.qeff[o * kHeadDim + i] = (float)(xr * mr - xi * mi);
+            p.qeff[o * kHeadDim + i + kBands] = (float)(xr * mi + xi * mr);
+            p.wts[o * kBands + i] =
+                (float)((1.0 - (double)p.R[row]) * ((double)p.qabs[row * kBands + i] - sqrt(xr * xr + xi * xi)));
+        }
+        if (i == 0 && p.unit_kmin) {
+            p.unit_kmin[u] = 0xffffffffu;
+            p.unit_kmax[u] = 0u;
+        }
+        return;
+    }
     double cr = 0.0, ci = 0.0, wa = 0.0;
     for (int g = 0; g < p.G; ++g) {
         const int64_t row = (int64_t)l * Hq + (int64_t)h * p.G + g;
@@ -96,12 +119,10 @@ __device__ void plan_sequences(const QueryParams& p) {
             p.len_ws[s] = len;
             const int nblk = (len + kBlockRows - 1) / kBlockRows;
             const bool compress = p.budget > 0;
-            const int scored = (compress && len <= p.budget) ? 0 : nblk;
+            const bool touched = !compress || len > p.trigger;
+            const int scored = touched ? nblk : 0;
             items = p.L * n_hg * ((scored + kChunkBlocks - 1) / kChunkBlocks);
-            if (compress) {
-                const int kept = len < p.budget ? len : p.budget;
-                nf = nblk - (kept + kBlockRows - 1) / kBlockRows;
-            }
+            if (compress && touched) nf = nblk - (p.budget + kBlockRows - 1) / kBlockRows;
         }
         int tot_i, tot_f;
         const int ex_i = block_exclusive_scan<kQueryThreads>(items, warp_tmp, tot_i);
@@ -117,6 +138,16 @@ __device__ void plan_sequences(const QueryParams& p) {
         p.item_off[p.S] = carry_items;
         p.freed_off[p.S] = carry_freed;
         if (p.freed_count) *p.freed_count = carry_freed;
+        if (p.fl_count) {
+            const int have = *p.fl_count;
+            if (have >= 0 && (int64_t)have + carry_freed <= (int64_t)p.fl_capacity) {
+                *p.fl_count = have + carry_freed;
+                *p.fl_base = have;
+            } else {
+                *p.fl_base = -1;
+                raise_flag(p.status, TRI_DEVFLAG_FREELIST);
+            }
+        }
         if (p.zero_words) {
             p.zero_words[0] = 0;
             p.zero_words[1] = 0;

@@ -32,6 +32,15 @@
 //    that range.
 //  * Every wait is bounded; on a timeout the CTA records TRI_DEVFLAG_TIMEOUT,
 //    lets its in-flight copies land and returns.
+//
+// Max over the GQA group (agg_heads = G): the G heads of a unit are scored
+// separately, s = max_g (qeff_g . K + sum_i w_{g,i} |K band i|).  A key is
+// shared by 64/BPL lanes with BPL bands each (BPL = 8, 8, 4, 2 for G = 1, 2,
+// 4, 8), so the 3*BPL*G coefficients of a lane stay within 48 registers; the
+// band magnitudes are computed once per key and reused by every head.  The
+// G partial sums are reduced with a butterfly that halves the live heads at
+// each step (a reduce-scatter over the key's lanes), then the lanes holding
+// different heads' totals exchange their maximum.
 #include "tri_device.cuh"
 #include "tri_internal.h"
 
@@ -81,6 +90,76 @@ __device__ __forceinline__ float key_score(const uint4 a, const uint4 b, const f
         nrm1 = fmaf(ww[2 * j + 1], sqrt_fast(fmaf(r1, r1, i1 * i1)), nrm1);
     }
     return (dot0 + dot1) + (nrm0 + nrm1);
+}
+
+// ---- max over the group -------------------------------------------------
+
+template <int G> struct MaxLayout;
+template <> struct MaxLayout<1> { static constexpr int kBpl = 8; };
+template <> struct MaxLayout<2> { static constexpr int kBpl = 8; };
+template <> struct MaxLayout<4> { static constexpr int kBpl = 4; };
+template <> struct MaxLayout<8> { static constexpr int kBpl = 2; };
+
+// BPL bf16 values of the real half (dims sub*BPL..) and of the imaginary
+// half (dims 64 + sub*BPL..) of a 256-byte key row.
+template <int BPL>
+__device__ __forceinline__ void load_bands(const uint8_t* row, int sub, float (&re)[BPL], float (&im)[BPL]) {
+    constexpr int W = BPL / 2;                 // 32-bit words per half
+    uint32_t a[W], b[W];
+    if constexpr (W == 4) {
+        const uint4 x = *reinterpret_cast<const uint4*>(row + sub * 16);
+        const uint4 y = *reinterpret_cast<const uint4*>(row + 128 + sub * 16);
+        a[0] = x.x; a[1] = x.y; a[2] = x.z; a[3] = x.w;
+        b[0] = y.x; b[1] = y.y; b[2] = y.z; b[3] = y.w;
+    } else if constexpr (W == 2) {
+        const uint2 x = *reinterpret_cast<const uint2*>(row + sub * 8);
+        const uint2 y = *reinterpret_cast<const uint2*>(row + 128 + sub * 8);
+        a[0] = x.x; a[1] = x.y;
+        b[0] = y.x; b[1] = y.y;
+    } else {
+        a[0] = *reinterpret_cast<const uint32_t*>(row + sub * 4);
+        b[0] = *reinterpret_cast<const uint32_t*>(row + 128 + sub * 4);
+    }
+#pragma unroll
+    for (int j = 0; j < W; ++j) {
+        re[2 * j] = bf16_lo(a[j]);
+        re[2 * j + 1] = bf16_hi(a[j]);
+        im[2 * j] = bf16_lo(b[j]);
+        im[2 * j + 1] = bf16_hi(b[j]);
+    }
+}
+
+// Butterfly over lane bit M and below: N live partial sums per lane; at each
+// step a lane keeps half of them (by its bit M) and adds its partner's copy of
+// that half.  Ends with v[0] = a full sum of one head.
+template <int N, int M, int G>
+__device__ __forceinline__ void scatter_heads(float (&v)[G], int lane) {
+    if constexpr (M >= 1) {
+        if constexpr (N > 1) {
+            constexpr int H = N / 2;
+            const bool upper = (lane & M) != 0;
+#pragma unroll
+            for (int j = 0; j < H; ++j) {
+                const float send = upper ? v[j] : v[j + H];
+                const float keep = upper ? v[j + H] : v[j];
+                v[j] = keep + __shfl_xor_sync(0xffffffffu, send, M);
+            }
+            scatter_heads<H, M / 2, G>(v, lane);
+        } else {
+            v[0] += __shfl_xor_sync(0xffffffffu, v[0], M);
+            scatter_heads<1, M / 2, G>(v, lane);
+        }
+    }
+}
+
+// Largest of the G head scores of the key shared by lanes of width LPK.
+template <int G, int LPK>
+__device__ __forceinline__ float group_max(float (&v)[G], int lane) {
+    scatter_heads<G, LPK / 2, G>(v, lane);
+    float r = v[0];
+#pragma unroll
+    for (int m = LPK / 2; m >= LPK / G; m >>= 1) r = fmaxf(r, __shfl_xor_sync(0xffffffffu, r, m));
+    return r;
 }
 
 __device__ void produce(const ScoreParams& p, uint8_t* tiles, uint64_t* full, uint64_t* empty, StageMeta* meta,
@@ -239,6 +318,98 @@ __device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t*
     }
 }
 
+template <int G>
+__device__ void consume_max(const ScoreParams& p, int warp, int lane, const uint8_t* tiles, uint64_t* full,
+                            uint64_t* empty, const StageMeta* meta, volatile int* abort_flag) {
+    constexpr int BPL = MaxLayout<G>::kBpl;
+    constexpr int LPK = kBands / BPL;          // lanes per key
+    constexpr int KPI = 32 / LPK;              // keys per warp step
+    const int HG = p.heads_per_tile;
+    const uint32_t stages = (uint32_t)p.stages;
+    const uint32_t stage_bytes = (uint32_t)HG * kTileBytes;
+    const int wph = kConsumerWarps / HG;
+    const int hig = warp / wph;
+    const int q0 = warp % wph;
+    const int sub = lane % LPK, kq = lane / LPK;
+    float qr[G][BPL], qi[G][BPL], ww[G][BPL];
+    int cur_unit = -1;
+    const uint64_t keep_pol = l2_policy_evict_last();
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    auto flush_range = [&]() {
+        const uint32_t lo = __reduce_min_sync(0xffffffffu, kmin);
+        const uint32_t hi = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0 && cur_unit >= 0 && lo <= hi) {
+            atomicMin(&p.unit_kmin[cur_unit], lo);
+            atomicMax(&p.unit_kmax[cur_unit], hi);
+        }
+        kmin = 0xffffffffu;
+        kmax = 0u;
+    };
+    for (uint32_t k = 0;; ++k) {
+        const uint32_t slot = k % stages;
+        if (!wait_or_abort(&full[slot], (k / stages) & 1u, abort_flag)) {
+            if (!*abort_flag) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
+            *abort_flag = 1;
+            return;
+        }
+        const StageMeta m = meta[slot];
+        if (m.kind == 2) {
+            flush_range();
+            return;
+        }
+        if (m.kind == 1) {
+            const int unit = m.unit0 + hig;
+            if (unit != cur_unit) {
+                flush_range();
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float* qe = p.qeff + ((int64_t)unit * G + g) * kHeadDim;
+                    const float* we = p.wts + ((int64_t)unit * G + g) * kBands;
+#pragma unroll
+                    for (int b = 0; b < BPL; ++b) {
+                        qr[g][b] = __ldg(qe + sub * BPL + b);
+                        qi[g][b] = __ldg(qe + kBands + sub * BPL + b);
+                        ww[g][b] = __ldg(we + sub * BPL + b);
+                    }
+                }
+                cur_unit = unit;
+            }
+            const uint8_t* tile = tiles + (size_t)slot * stage_bytes + (size_t)hig * kTileBytes;
+            float* out = p.scores + (int64_t)unit * p.score_stride + m.t0;
+            for (int q = q0; q < kBlockRows / KPI; q += wph) {
+                const int row = q * KPI + kq;
+                float re[BPL], im[BPL], nrm[BPL];
+                load_bands<BPL>(tile + row * 256, sub, re, im);
+#pragma unroll
+                for (int b = 0; b < BPL; ++b) nrm[b] = sqrt_fast(fmaf(re[b], re[b], im[b] * im[b]));
+                float v[G];
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    float d0 = 0.f, d1 = 0.f;
+#pragma unroll
+                    for (int b = 0; b < BPL; ++b) {
+                        d0 = fmaf(qr[g][b], re[b], d0);
+                        d1 = fmaf(qi[g][b], im[b], d1);
+                        d0 = fmaf(ww[g][b], nrm[b], d0);
+                    }
+                    v[g] = d0 + d1;
+                }
+                const float acc = group_max<G, LPK>(v, lane);
+                if (sub == 0 && row < m.nrows) {
+                    store_with_policy(out + row, acc, keep_pol);
+                    const uint32_t key = order_key(acc);
+                    kmin = min(kmin, key);
+                    kmax = max(kmax, key);
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+}
+
+// AGG = 0: folded group mean; AGG = G: max over the G heads of the group.
+template <int AGG>
 __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScoreParams p) {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t stages = (uint32_t)p.stages;
@@ -263,7 +434,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
         if (lane == 0) produce(p, tiles, full, empty, meta, abort_flag);
         return;
     }
-    consume(p, warp, lane, tiles, full, empty, meta, abort_flag);
+    if constexpr (AGG == 0)
+        consume(p, warp, lane, tiles, full, empty, meta, abort_flag);
+    else
+        consume_max<AGG>(p, warp, lane, tiles, full, empty, meta, abort_flag);
 }
 
 size_t score_smem_bytes(int HG, int stages) {
@@ -286,12 +460,21 @@ cudaError_t launch_score(const ScoreParams& p_in, int max_items, int num_sms, cu
     if (stages < 2) stages = 2;
     p.stages = stages;
     const size_t smem = score_smem_bytes(p.heads_per_tile, stages);
-    cudaError_t e = cudaFuncSetAttribute(score_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    void (*kernel)(const ScoreParams);
+    switch (p.agg_heads) {
+        case 0: kernel = score_kernel<0>; break;
+        case 1: kernel = score_kernel<1>; break;
+        case 2: kernel = score_kernel<2>; break;
+        case 4: kernel = score_kernel<4>; break;
+        case 8: kernel = score_kernel<8>; break;
+        default: return cudaErrorInvalidValue;
+    }
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     int grid = num_sms * 2;
     if (max_items < grid) grid = max_items;
     if (grid < 1) grid = 1;
-    return launch_kernel(score_kernel, dim3(grid), dim3(kScoreThreads), smem, stream, pdl, p);
+    return launch_kernel(kernel, dim3(grid), dim3(kScoreThreads), smem, stream, pdl, p);
 }
 
 }  // namespace tri

@@ -33,14 +33,16 @@ int scratch_rows_for(const tri_kv_desc* d, int budget) {
     return (int)(rows < 64 ? 64 : (rows > (1 << 24) ? (1 << 24) : rows));
 }
 
-// Workspace of a step with budget `budget` (0: the score-only part).
-WsLayout ws_layout(const tri_kv_desc* d, int budget) {
+// Workspace of a step with budget `budget` (0: the score-only part);
+// per_head: G coefficient sets per unit (max over the group).
+WsLayout ws_layout(const tri_kv_desc* d, int budget, bool per_head = false) {
     const size_t U = (size_t)d->S * d->L * d->Hkv;
+    const size_t sets = U * (per_head ? (size_t)d->G : 1);
     const size_t max_len = (size_t)d->max_blocks * kBlockRows;
     WsLayout w;
     size_t off = 0;
-    w.qeff = off;      off = align_up(off + U * kHeadDim * sizeof(float));
-    w.wts = off;       off = align_up(off + U * kBands * sizeof(float));
+    w.qeff = off;      off = align_up(off + sets * kHeadDim * sizeof(float));
+    w.wts = off;       off = align_up(off + sets * kBands * sizeof(float));
     w.len_ws = off;    off = align_up(off + (size_t)d->S * sizeof(int32_t));
     w.item_off = off;  off = align_up(off + ((size_t)d->S + 1) * sizeof(int32_t));
     w.freed_off = off; off = align_up(off + ((size_t)d->S + 1) * sizeof(int32_t));
@@ -50,7 +52,7 @@ WsLayout ws_layout(const tri_kv_desc* d, int budget) {
     w.idx = off;       off = align_up(off + U * (size_t)(budget > 0 ? budget : 0) * sizeof(int32_t));
     w.scratch_rows = scratch_rows_for(d, budget);
     const size_t per_unit = budget > 0 ? 1 : 0;
-    w.words = off;     off = align_up(off + 2 * sizeof(int32_t) * per_unit);
+    w.words = off;     off = align_up(off + 4 * sizeof(int32_t) * per_unit);   // scratch rows used, 0, free-list base
     w.info = off;      off = align_up(off + U * 4 * sizeof(int32_t) * per_unit);
     w.owner = off;     off = align_up(off + (size_t)w.scratch_rows * 2 * sizeof(int32_t));
     w.scratch = off;   off = align_up(off + (size_t)w.scratch_rows * 2 * kHeadDim * 2);
@@ -98,9 +100,34 @@ tri_status check_budget(int budget, int window) {
     return TRI_OK;
 }
 
-tri_status check_workspace(const tri_kv_desc* d, const void* ws, size_t ws_bytes, int budget) {
+tri_status check_workspace(const tri_kv_desc* d, const void* ws, size_t ws_bytes, int budget,
+                           bool per_head = false) {
     if (ws == nullptr || ((uintptr_t)ws % kWsAlign) != 0) return TRI_ERR_WORKSPACE;
-    if (ws_bytes < ws_layout(d, budget).total) return TRI_ERR_WORKSPACE;
+    if (ws_bytes < ws_layout(d, budget, per_head).total) return TRI_ERR_WORKSPACE;
+    return TRI_OK;
+}
+
+tri_status check_aggregate(int aggregate, int G) {
+    if (aggregate == TRI_AGG_MEAN) return TRI_OK;
+    if (aggregate != TRI_AGG_MAX) return TRI_ERR_INVALID;
+    return (G == 1 || G == 2 || G == 4 || G == 8) ? TRI_OK : TRI_ERR_UNSUPPORTED;
+}
+
+// Options of a selection / step; G for the aggregate check (0: not checked).
+tri_status check_options(const tri_step_options* o, int G) {
+    if (o == nullptr) return TRI_ERR_INVALID;
+    tri_status st = check_budget(o->budget, o->window);
+    if (st != TRI_OK) return st;
+    if (o->sinks < 0 || o->trigger < 0 || (int64_t)o->sinks + o->window > o->budget) return TRI_ERR_INVALID;
+    return G > 0 ? check_aggregate(o->aggregate, G) : TRI_OK;
+}
+
+int effective_trigger(const tri_step_options& o) { return o.trigger > o.budget ? o.trigger : o.budget; }
+
+tri_status check_free_list(const tri_free_list* fl) {
+    if (fl == nullptr) return TRI_OK;
+    if (!fl->ids || !fl->count || fl->capacity < 0 || !aligned(fl->ids, 4) || !aligned(fl->count, 4))
+        return TRI_ERR_INVALID;
     return TRI_OK;
 }
 
@@ -163,6 +190,7 @@ ScoreParams make_score_params(const tri_kv_desc* d, const uint8_t* ws, const WsL
     s.S = d->S;
     s.max_blocks = d->max_blocks;
     s.heads_per_tile = score_heads_per_tile(d->Hkv);
+    s.agg_heads = 0;
     return s;
 }
 
@@ -239,20 +267,35 @@ size_t tri_workspace_size(const tri_kv_desc* desc, int budget) {
     return ws_layout(desc, budget).total;
 }
 
+size_t tri_workspace_size_ex(const tri_kv_desc* desc, const tri_step_options* opt) {
+    if (check_desc(desc) != TRI_OK || check_options(opt, desc->G) != TRI_OK) return 0;
+    return ws_layout(desc, opt->budget, opt->aggregate == TRI_AGG_MAX).total;
+}
+
 tri_status tri_score(const tri_kv_desc* desc, const float* qbar, const float* qabs, const float* R,
                      double rope_base, const int32_t* deltas, int n_deltas, float* scores, void* workspace,
                      size_t ws_bytes, cudaStream_t stream) {
+    return tri_score_ex(desc, qbar, qabs, R, rope_base, deltas, n_deltas, TRI_AGG_MEAN, scores, workspace,
+                        ws_bytes, stream);
+}
+
+tri_status tri_score_ex(const tri_kv_desc* desc, const float* qbar, const float* qabs, const float* R,
+                        double rope_base, const int32_t* deltas, int n_deltas, int aggregate, float* scores,
+                        void* workspace, size_t ws_bytes, cudaStream_t stream) {
     tri_status st = check_desc(desc);
     if (st != TRI_OK) return st;
     if ((st = check_stats(qbar, qabs, R)) != TRI_OK) return st;
     if ((st = check_query_args(rope_base, deltas, n_deltas)) != TRI_OK) return st;
+    if ((st = check_aggregate(aggregate, desc->G)) != TRI_OK) return st;
     if (!scores || !aligned(scores, 4)) return TRI_ERR_INVALID;
-    if ((st = check_workspace(desc, workspace, ws_bytes, 0)) != TRI_OK) return st;
+    const bool per_head = aggregate == TRI_AGG_MAX;
+    if ((st = check_workspace(desc, workspace, ws_bytes, 0, per_head)) != TRI_OK) return st;
     if (desc->S == 0) return TRI_OK;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const WsLayout w = ws_layout(desc, 0);
+    const WsLayout w = ws_layout(desc, 0, per_head);
     QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
                                       reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
+    q.per_head = per_head ? 1 : 0;
     q.do_plan = 1;
     q.budget = 0;
     q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
@@ -263,22 +306,31 @@ tri_status tri_score(const tri_kv_desc* desc, const float* qbar, const float* qa
     q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     ScoreParams sp = make_score_params(desc, ws, w, scores, (int64_t)desc->max_blocks * kBlockRows);
+    sp.agg_heads = per_head ? desc->G : 0;
     return cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream));
 }
 
 tri_status tri_select_topk(const tri_kv_desc* desc, const float* scores, int budget, int window, int32_t* idx,
                            int32_t* kept, cudaStream_t stream) {
+    const tri_step_options o = {budget, window, 0, 0, TRI_AGG_MEAN};
+    return tri_select_topk_ex(desc, scores, &o, idx, kept, stream);
+}
+
+tri_status tri_select_topk_ex(const tri_kv_desc* desc, const float* scores, const tri_step_options* opt,
+                              int32_t* idx, int32_t* kept, cudaStream_t stream) {
     tri_status st = check_desc(desc);
     if (st != TRI_OK) return st;
-    if ((st = check_budget(budget, window)) != TRI_OK) return st;
+    if ((st = check_options(opt, 0)) != TRI_OK) return st;
     if (!scores || !idx || !kept || !aligned(scores, 16) || !aligned(idx, 4) || !aligned(kept, 4))
         return TRI_ERR_INVALID;
     if (desc->S == 0) return TRI_OK;
     EvictParams e = make_evict_params(desc);
     e.scores = scores;
     e.lens = desc->seq_len;
-    e.budget = budget;
-    e.window = window;
+    e.budget = opt->budget;
+    e.window = opt->window;
+    e.sinks = opt->sinks;
+    e.trigger = effective_trigger(*opt);
     e.idx_out = idx;
     e.kept_out = kept;
     e.do_select = 1;
@@ -299,6 +351,7 @@ tri_status tri_compact_kv(tri_kv_desc* desc, const int32_t* idx, const int32_t* 
     EvictParams e = make_evict_params(desc);
     e.lens = desc->seq_len;
     e.budget = budget;
+    e.trigger = budget;
     e.idx_in = idx;
     e.kept_in = kept;
     e.do_select = 0;
@@ -307,6 +360,7 @@ tri_status tri_compact_kv(tri_kv_desc* desc, const int32_t* idx, const int32_t* 
     MoveParams mv = make_move_params(desc, idx, budget);
     mv.lens = desc->seq_len;
     mv.kept = kept;
+    mv.trigger = budget;
     if ((st = cuda_status(launch_move(mv, device_sm_count(), stream))) != TRI_OK) return st;
     FinalizeParams f{};
     f.seq_len = desc->seq_len;
@@ -324,17 +378,33 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
                              double rope_base, const int32_t* deltas, int n_deltas, int budget, int window,
                              int32_t* freed_ids, int32_t* freed_count, int32_t* idx_out, void* workspace,
                              size_t ws_bytes, const tri_phase_events* events, cudaStream_t stream) {
+    if (!freed_ids || !freed_count) return TRI_ERR_INVALID;
+    const tri_step_options o = {budget, window, 0, 0, TRI_AGG_MEAN};
+    return tri_compress_step_ex(desc, qbar, qabs, R, rope_base, deltas, n_deltas, &o, nullptr, freed_ids,
+                                freed_count, idx_out, workspace, ws_bytes, events, stream);
+}
+
+tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const float* qabs, const float* R,
+                                double rope_base, const int32_t* deltas, int n_deltas, const tri_step_options* opt,
+                                const tri_free_list* free_list, int32_t* freed_ids, int32_t* freed_count,
+                                int32_t* idx_out, void* workspace, size_t ws_bytes, const tri_phase_events* events,
+                                cudaStream_t stream) {
     tri_status st = check_desc(desc);
     if (st != TRI_OK) return st;
     if ((st = check_stats(qbar, qabs, R)) != TRI_OK) return st;
     if ((st = check_query_args(rope_base, deltas, n_deltas)) != TRI_OK) return st;
-    if ((st = check_budget(budget, window)) != TRI_OK) return st;
-    if (!freed_ids || !freed_count || !aligned(freed_ids, 4) || !aligned(freed_count, 4)) return TRI_ERR_INVALID;
+    if ((st = check_options(opt, desc->G)) != TRI_OK) return st;
+    if ((st = check_free_list(free_list)) != TRI_OK) return st;
+    if ((freed_ids == nullptr) != (freed_count == nullptr)) return TRI_ERR_INVALID;
+    if (!freed_ids && !free_list) return TRI_ERR_INVALID;
+    if ((freed_ids && !aligned(freed_ids, 4)) || (freed_count && !aligned(freed_count, 4))) return TRI_ERR_INVALID;
     if (idx_out && !aligned(idx_out, 4)) return TRI_ERR_INVALID;
-    if ((st = check_workspace(desc, workspace, ws_bytes, budget)) != TRI_OK) return st;
+    const int budget = opt->budget;
+    const bool per_head = opt->aggregate == TRI_AGG_MAX;
+    if ((st = check_workspace(desc, workspace, ws_bytes, budget, per_head)) != TRI_OK) return st;
     if (events) record(events->start, stream);
     if (desc->S == 0) {
-        st = cuda_status(cudaMemsetAsync(freed_count, 0, sizeof(int32_t), stream));
+        st = freed_count ? cuda_status(cudaMemsetAsync(freed_count, 0, sizeof(int32_t), stream)) : TRI_OK;
         if (events) {
             record(events->after_query, stream);
             record(events->after_score, stream);
@@ -343,11 +413,14 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
         return st;
     }
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    const WsLayout w = ws_layout(desc, budget);
+    const WsLayout w = ws_layout(desc, budget, per_head);
+    const int trigger = effective_trigger(*opt);
     QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
                                       reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
+    q.per_head = per_head ? 1 : 0;
     q.do_plan = 1;
     q.budget = budget;
+    q.trigger = trigger;
     q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
     q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
     q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
@@ -355,6 +428,11 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     q.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
     q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
     q.zero_words = reinterpret_cast<int32_t*>(ws + w.words);
+    if (free_list) {
+        q.fl_count = free_list->count;
+        q.fl_capacity = free_list->capacity;
+        q.fl_base = reinterpret_cast<int32_t*>(ws + w.words) + 2;
+    }
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     if (events) record(events->after_query, stream);
 
@@ -363,6 +441,7 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     const bool pdl = events == nullptr;
     float* scores = reinterpret_cast<float*>(ws + w.scores);
     ScoreParams sp = make_score_params(desc, ws, w, scores, (int64_t)desc->max_blocks * kBlockRows);
+    sp.agg_heads = per_head ? desc->G : 0;
     if ((st = cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream, pdl))) != TRI_OK)
         return st;
     if (events) record(events->after_score, stream);
@@ -373,7 +452,9 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     e.unit_kmax = reinterpret_cast<const uint32_t*>(ws + w.kmax);
     e.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
     e.budget = budget;
-    e.window = window;
+    e.window = opt->window;
+    e.sinks = opt->sinks;
+    e.trigger = trigger;
     e.idx_out = reinterpret_cast<int32_t*>(ws + w.idx);
     e.idx_copy = idx_out;
     e.do_select = 1;
@@ -381,6 +462,10 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     e.seq_len_out = desc->seq_len;
     e.freed_off = reinterpret_cast<const int32_t*>(ws + w.freed_off);
     e.freed_ids = freed_ids;
+    if (free_list) {
+        e.fl_ids = free_list->ids;
+        e.fl_base = reinterpret_cast<const int32_t*>(ws + w.words) + 2;
+    }
     e.scratch_used = reinterpret_cast<int32_t*>(ws + w.words);
     e.unit_info = reinterpret_cast<int32_t*>(ws + w.info);
     e.scratch_owner = reinterpret_cast<int32_t*>(ws + w.owner);
@@ -389,6 +474,7 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     MoveParams mv = make_move_params(desc, reinterpret_cast<const int32_t*>(ws + w.idx), budget);
     mv.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
     mv.kept = nullptr;
+    mv.trigger = trigger;
     mv.unit_info = reinterpret_cast<const int32_t*>(ws + w.info);
     mv.scratch = ws + w.scratch;
     mv.scratch_owner = reinterpret_cast<const int32_t*>(ws + w.owner);
@@ -400,6 +486,29 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
     if ((st = cuda_status(launch_move(mv, device_sm_count(), stream, pdl))) != TRI_OK) return st;
     if (events) record(events->after_evict, stream);
     return TRI_OK;
+}
+
+tri_status tri_reserve_blocks(const tri_kv_desc* desc, int32_t* block_table, const int32_t* n_new,
+                              const tri_free_list* free_list, cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if (!block_table || block_table != desc->block_table || !n_new || !aligned(n_new, 4) || !free_list)
+        return TRI_ERR_INVALID;
+    if ((st = check_free_list(free_list)) != TRI_OK) return st;
+    if ((int64_t)desc->S * desc->max_blocks > INT_MAX) return TRI_ERR_INVALID;
+    if (desc->S == 0) return TRI_OK;
+    ReserveParams r{};
+    r.seq_len = desc->seq_len;
+    r.n_new = n_new;
+    r.block_table = block_table;
+    r.S = desc->S;
+    r.max_blocks = desc->max_blocks;
+    r.num_blocks = desc->num_blocks;
+    r.fl_ids = free_list->ids;
+    r.fl_count = free_list->count;
+    r.fl_capacity = free_list->capacity;
+    r.status = desc->status;
+    return cuda_status(launch_reserve(r, stream));
 }
 
 tri_status tri_sync_status(int32_t* status, cudaStream_t stream) {
@@ -414,6 +523,7 @@ tri_status tri_sync_status(int32_t* status, cudaStream_t stream) {
     }
     if (h & TRI_DEVFLAG_BOUNDS) return TRI_ERR_DEVICE_BOUNDS;
     if (h & TRI_DEVFLAG_TIMEOUT) return TRI_ERR_TIMEOUT;
+    if (h & TRI_DEVFLAG_FREELIST) return TRI_ERR_FREELIST;
     if (h & TRI_DEVFLAG_NONFINITE) return TRI_ERR_NONFINITE;
     return TRI_OK;
 }
@@ -428,6 +538,7 @@ const char* tri_status_string(tri_status s) {
         case TRI_ERR_TIMEOUT: return "bounded device wait timed out";
         case TRI_ERR_NONFINITE: return "NaN score";
         case TRI_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+        case TRI_ERR_FREELIST: return "device free list had too few entries or too little room";
         default: return "unknown status";
     }
 }

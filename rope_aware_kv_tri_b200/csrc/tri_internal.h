@@ -43,14 +43,16 @@ struct QueryParams {
     double base;
     int n_deltas;
     int32_t deltas[TRI_MAX_DELTAS];
-    float* qeff;              // [U][D]
-    float* wts;               // [U][D/2]
+    float* qeff;              // [U][D], or [U][G][D] per head (aggregate == max)
+    float* wts;               // [U][D/2], or [U][G][D/2]
     int L, Hkv, G, S;
+    int per_head;             // 1: per-head coefficients (max over the group), 0: group mean
     // plan (last block of the grid when do_plan != 0)
     int do_plan;
     const int32_t* seq_len;   // [S]
     int max_blocks;
     int budget;               // 0: plan every sequence (score only)
+    int trigger;              // compress sequences with len > trigger (>= budget)
     int heads_per_tile;       // HG
     int32_t* len_ws;          // [S]
     int32_t* item_off;        // [S+1]
@@ -59,6 +61,9 @@ struct QueryParams {
     uint32_t* unit_kmin;      // [U] set to the largest key (min accumulator) or null
     uint32_t* unit_kmax;      // [U] set to 0 (max accumulator) or null
     int32_t* zero_words;      // [2] set to 0 by the plan CTA, or null
+    int32_t* fl_count;        // free list to push the freed ids on, or null
+    int fl_capacity;
+    int32_t* fl_base;         // [1] out: first list entry of this step's ids, -1 if no room
     int32_t* status;
 };
 cudaError_t launch_query(const QueryParams& p, cudaStream_t stream);
@@ -78,6 +83,7 @@ struct ScoreParams {
     int32_t* status;
     int L, Hkv, num_blocks, S, max_blocks;
     int heads_per_tile;       // HG, divides 8 and Hkv
+    int agg_heads;            // 0: folded group mean; G: max over G per-head scores
     int stages;
 };
 int score_heads_per_tile(int Hkv);
@@ -91,6 +97,8 @@ struct EvictParams {
     const uint32_t* unit_kmax;
     const int32_t* lens;       // lengths the unit works from
     int budget, window;
+    int sinks;                 // leading slots always kept
+    int trigger;               // units with len <= trigger keep every slot (>= budget)
     int32_t* idx_out;          // [U][budget] or null
     int32_t* idx_copy;         // [U][budget] second copy of the kept slots, or null
     int32_t* kept_out;         // [S] or null
@@ -105,6 +113,8 @@ struct EvictParams {
     int32_t* seq_len_out;      // or null
     const int32_t* freed_off;  // [S+1] or null
     int32_t* freed_ids;        // or null
+    int32_t* fl_ids;           // free list entries, or null
+    const int32_t* fl_base;    // [1] where this step's ids start in fl_ids (-1: none)
     int32_t* status;
     // step plans (null outside tri_compress_step)
     int32_t* scratch_used;     // [1] rows of the scratch handed out, 0 at launch
@@ -119,7 +129,8 @@ struct MoveParams {
     const int32_t* idx;        // [U][budget] kept slots, ascending
     int budget;
     const int32_t* lens;       // [S] lengths before the step
-    const int32_t* kept;       // [S], or null: min(len, budget) for len > budget, else untouched
+    const int32_t* kept;       // [S], or null: budget for len > trigger, else untouched
+    int trigger;               // (>= budget) used when kept is null
     uint8_t* k_pool;
     uint8_t* v_pool;
     const int32_t* block_table;
@@ -145,6 +156,19 @@ struct FinalizeParams {
     int32_t* status;
 };
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t stream);
+
+// Pop blocks for n_new[s] more slots per sequence from a device free list.
+struct ReserveParams {
+    const int32_t* seq_len;
+    const int32_t* n_new;
+    int32_t* block_table;
+    int S, max_blocks, num_blocks;
+    int32_t* fl_ids;
+    int32_t* fl_count;
+    int fl_capacity;
+    int32_t* status;
+};
+cudaError_t launch_reserve(const ReserveParams& p, cudaStream_t stream);
 
 // ------------------------------------------------------------- calibrate
 cudaError_t launch_calibrate(const float* q, int N, int L, int Hq, float* qbar, float* qabs, float* R,

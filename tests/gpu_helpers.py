@@ -72,12 +72,13 @@ def unit_rows(pool: torch.Tensor, table_row: List[int], length: int, l: int, h: 
     return pool[l, blocks, h].reshape(nb * 16, pool.shape[-1])[:length]
 
 
-def oracle_unit_scores(wl, keys: torch.Tensor, stats, s: int, l: int, h: int) -> np.ndarray:
+def oracle_unit_scores(wl, keys: torch.Tensor, stats, s: int, l: int, h: int,
+                       aggregate: str = "mean") -> np.ndarray:
     G = wl.cfg.G
     qb, qa, r = stats
     sl = slice(h * G, (h + 1) * G)
     return oracle.unit_scores(keys.double().cpu().numpy(), qb[l, sl], qa[l, sl], r[l, sl],
-                              int(wl.cur_pos[s].item()), wl.deltas, wl.cfg.base)
+                              int(wl.cur_pos[s].item()), wl.deltas, wl.cfg.base, aggregate=aggregate)
 
 
 def check_scores(s_gpu: np.ndarray, s_ref: np.ndarray, tol: float = SCORE_TOL) -> float:
@@ -94,10 +95,10 @@ def check_scores(s_gpu: np.ndarray, s_ref: np.ndarray, tol: float = SCORE_TOL) -
 
 
 def check_selection(idx_gpu: np.ndarray, s_ref: np.ndarray, length: int, budget: int, window: int,
-                    tol: float = SCORE_TOL) -> int:
+                    tol: float = SCORE_TOL, sinks: int = 0) -> int:
     """Assert the index rule against the oracle's float64 scores; returns the
     number of kept slots that differ (all of them inside the cut band)."""
-    ref = oracle.select(s_ref, length, budget, window)
+    ref = oracle.select(s_ref, length, budget, window, sinks)
     idx_gpu = np.asarray(idx_gpu, dtype=np.int64)
     assert idx_gpu.shape == ref.shape, (idx_gpu.shape, ref.shape)
     assert np.all(np.diff(idx_gpu) > 0), "kept slots not strictly ascending"
@@ -106,15 +107,17 @@ def check_selection(idx_gpu: np.ndarray, s_ref: np.ndarray, length: int, budget:
         return 0
     cand, take = length - window, budget - window
     assert np.array_equal(idx_gpu[take:], np.arange(cand, length)), "recent window not kept"
+    assert np.array_equal(idx_gpu[:sinks], np.arange(sinks)), "sink slots not kept"
+    take -= sinks
     if take == 0:
         return 0
-    order = sorted(range(cand), key=lambda t: (-s_ref[t], t))
+    order = sorted(range(sinks, cand), key=lambda t: (-s_ref[t], t))
     s_cut = s_ref[order[take - 1]]
     m_u = float(np.mean(np.abs(s_ref)))
     tau = tol * max(abs(s_cut), m_u)
     diff = set(idx_gpu.tolist()) ^ set(ref.tolist())
     for t in diff:
-        assert t < cand and abs(s_ref[t] - s_cut) <= tau, (
+        assert sinks <= t < cand and abs(s_ref[t] - s_cut) <= tau, (
             f"slot {t} differs with score {s_ref[t]} far from the cut {s_cut} (tau {tau})")
     return len(diff)
 

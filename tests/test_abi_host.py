@@ -39,7 +39,7 @@ def test_exports_every_declared_function(lib):
 
 def test_status_strings(lib):
     assert tri.tri_status_string(0) == "ok"
-    for code in range(1, 8):
+    for code in range(1, 9):
         assert tri.tri_status_string(code) not in ("ok", "unknown status")
     assert tri.tri_status_string(99) == "unknown status"
 
@@ -135,3 +135,87 @@ def test_binding_refuses_cpu_tensors(lib):
     with pytest.raises(ValueError):
         tri.tri_calibrate_centers(torch.zeros(2, 1, 1, 128), torch.zeros(1, 1, 128), torch.zeros(1, 1, 64),
                                   torch.zeros(1, 1))
+
+
+def _opts(**kw):
+    o = dict(budget=64, window=8, sinks=0, trigger=0, aggregate=tri.TRI_AGG_MEAN)
+    o.update(kw)
+    return tri.TriStepOptions(**o)
+
+
+def _step_ex(lib, desc, opt, free_list=None, freed=FAKE, count=FAKE, ws_bytes=None):
+    arr = (ctypes.c_int32 * 3)(1, 2, 4)
+    if ws_bytes is None:
+        ws_bytes = lib.tri_workspace_size_ex(ctypes.byref(desc), ctypes.byref(opt)) or (1 << 40)
+    return lib.tri_compress_step_ex(ctypes.byref(desc), FAKE, FAKE, FAKE, 1e4, arr, 3,
+                                    ctypes.byref(opt) if opt is not None else None,
+                                    ctypes.byref(free_list) if free_list is not None else None,
+                                    freed, count, None, FAKE, ws_bytes, None, None)
+
+
+def test_workspace_size_ex(lib):
+    d = _desc()
+    mean = lib.tri_workspace_size_ex(ctypes.byref(d), ctypes.byref(_opts()))
+    assert mean == lib.tri_workspace_size(ctypes.byref(d), 64)
+    mx = lib.tri_workspace_size_ex(ctypes.byref(d), ctypes.byref(_opts(aggregate=tri.TRI_AGG_MAX)))
+    U = 2 * 2 * 8
+    assert mx >= mean + (4 - 1) * U * 192 * 4 - 512          # G = 4 coefficient sets per unit
+    assert lib.tri_workspace_size_ex(ctypes.byref(_desc(G=3)), ctypes.byref(_opts(aggregate=1))) == 0
+    assert lib.tri_workspace_size_ex(ctypes.byref(d), ctypes.byref(_opts(sinks=60))) == 0
+    assert lib.tri_workspace_size_ex(ctypes.byref(d), None) == 0
+
+
+@pytest.mark.parametrize("opt,expect", [
+    (None, tri.TRI_ERR_INVALID),
+    (dict(sinks=-1), tri.TRI_ERR_INVALID),
+    (dict(sinks=57), tri.TRI_ERR_INVALID),                 # sinks + window > budget
+    (dict(trigger=-5), tri.TRI_ERR_INVALID),
+    (dict(aggregate=7), tri.TRI_ERR_INVALID),
+    (dict(budget=0), tri.TRI_ERR_INVALID),
+    (dict(budget=tri.TRI_MAX_BUDGET + 1, window=0), tri.TRI_ERR_UNSUPPORTED),
+])
+def test_step_ex_rejects_options(lib, opt, expect):
+    o = None if opt is None else _opts(**opt)
+    assert _step_ex(lib, _desc(), o, ws_bytes=1 << 40) == expect
+
+
+def test_step_ex_rejects_max_for_odd_group(lib):
+    assert _step_ex(lib, _desc(G=3), _opts(aggregate=tri.TRI_AGG_MAX), ws_bytes=1 << 40) == tri.TRI_ERR_UNSUPPORTED
+
+
+def test_step_ex_output_rules(lib):
+    d = _desc()
+    # neither freed ids nor a free list
+    assert _step_ex(lib, d, _opts(), freed=None, count=None) == tri.TRI_ERR_INVALID
+    # freed ids without a count
+    assert _step_ex(lib, d, _opts(), freed=FAKE, count=None) == tri.TRI_ERR_INVALID
+    bad = tri.TriFreeList(ids=None, count=FAKE, capacity=10)
+    assert _step_ex(lib, d, _opts(), free_list=bad) == tri.TRI_ERR_INVALID
+    neg = tri.TriFreeList(ids=FAKE, count=FAKE, capacity=-1)
+    assert _step_ex(lib, d, _opts(), free_list=neg) == tri.TRI_ERR_INVALID
+    # the max workspace is larger than the mean one
+    mean_bytes = lib.tri_workspace_size_ex(ctypes.byref(d), ctypes.byref(_opts()))
+    assert _step_ex(lib, d, _opts(aggregate=tri.TRI_AGG_MAX), ws_bytes=mean_bytes) == tri.TRI_ERR_WORKSPACE
+
+
+def test_select_ex_and_score_ex_reject(lib):
+    d = _desc()
+    assert lib.tri_select_topk_ex(ctypes.byref(d), FAKE, ctypes.byref(_opts(sinks=57)), FAKE, FAKE,
+                                  None) == tri.TRI_ERR_INVALID
+    assert lib.tri_select_topk_ex(ctypes.byref(d), FAKE + 4, ctypes.byref(_opts()), FAKE, FAKE,
+                                  None) == tri.TRI_ERR_INVALID      # scores not 16-byte aligned
+    arr = (ctypes.c_int32 * 1)(1)
+    assert lib.tri_score_ex(ctypes.byref(d), FAKE, FAKE, FAKE, 1e4, arr, 1, 5, FAKE, FAKE, 1 << 40,
+                            None) == tri.TRI_ERR_INVALID
+    assert lib.tri_score_ex(ctypes.byref(_desc(G=6)), FAKE, FAKE, FAKE, 1e4, arr, 1, tri.TRI_AGG_MAX, FAKE,
+                            FAKE, 1 << 40, None) == tri.TRI_ERR_UNSUPPORTED
+
+
+def test_reserve_rejects(lib):
+    d = _desc()
+    fl = tri.TriFreeList(ids=FAKE, count=FAKE, capacity=10)
+    assert lib.tri_reserve_blocks(ctypes.byref(d), FAKE + 64, FAKE, ctypes.byref(fl), None) == tri.TRI_ERR_INVALID
+    assert lib.tri_reserve_blocks(ctypes.byref(d), FAKE, FAKE, None, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_reserve_blocks(ctypes.byref(d), FAKE, None, ctypes.byref(fl), None) == tri.TRI_ERR_INVALID
+    assert lib.tri_reserve_blocks(ctypes.byref(_desc(D=64)), FAKE, FAKE, ctypes.byref(fl),
+                                  None) == tri.TRI_ERR_UNSUPPORTED
