@@ -266,6 +266,108 @@ def compress_unit(keys_f64: np.ndarray, k_rows: np.ndarray, v_rows: np.ndarray,
     return s, idx, compact_rows(k_rows, idx), compact_rows(v_rows, idx)
 
 
+# ----------------------------------------------------------------------------
+# Variant: scores from the centres alone, as a table over the distance
+# [Digest] "Core Mechanism" (the trigonometric series of the distance,
+# evaluated as lookups indexed by relative position) and "Key Concepts",
+# Trigonometric Distance Preference (after rotation the centres' dot product
+# depends on the query-key distance only).
+#
+# Reading: the table is the trigonometric term with the key's own rotated
+# band replaced by its head's rotated key centre kbar (calibrated from
+# pre-rotation keys like the query centre).  The norm term of the centres,
+# (1 - R) sum_i (A_i - |qbar_i|) |kbar_i|, is the same for every key of a unit
+# and cannot change its ranking, so the table leaves it out.  A key's score
+# is f(p - pos_t), pos_t the position the key was cached at; after a
+# compaction slots no longer equal positions, so positions travel with the
+# rows.
+# ----------------------------------------------------------------------------
+
+def distance_series(qbar_g: np.ndarray, kbar: np.ndarray, deltas: Sequence[int], base: float,
+                    max_dist: int) -> np.ndarray:
+    """f_g(dist) for dist = 0 .. max_dist, one query head g against a key
+    centre:
+      logit(p + delta, t) = sum_i Re( qbar_i e^{j theta_i (p+delta)} conj(kbar_i e^{j theta_i t}) )
+                          = sum_i Re( qbar_i conj(kbar_i) e^{j theta_i (dist + delta)} ),  dist = p - t,
+    averaged uniformly over the offsets delta."""
+    qb = as_bands(np.asarray(qbar_g, dtype=np.float64))
+    kb = as_bands(np.asarray(kbar, dtype=np.float64))
+    theta = rope_frequencies(qbar_g.shape[-1], base)
+    a = qb * np.conj(kb)
+    dist = np.arange(int(max_dist) + 1, dtype=np.float64)
+    out = np.zeros(dist.shape[0], dtype=np.float64)
+    for d in deltas:
+        phase = np.exp(1j * theta[None, :] * (dist[:, None] + float(int(d))))
+        out += (a[None, :] * phase).real.sum(axis=-1)
+    return out / len(deltas)
+
+
+def distance_table(qbar: np.ndarray, kbar: np.ndarray, deltas: Sequence[int], base: float,
+                   max_dist: int, aggregate: str = "mean") -> np.ndarray:
+    """The table of one (layer, KV head): its G query heads' series
+    (qbar [G, D], kbar [D]) combined per distance by mean (the method's
+    reading) or max (the variant)."""
+    G = qbar.shape[0]
+    per_head = [distance_series(qbar[g], kbar, deltas, base, max_dist) for g in range(G)]
+    if aggregate == "mean":
+        total = np.zeros_like(per_head[0])
+        for f in per_head:
+            total += f
+        return total / G
+    if aggregate == "max":
+        best = per_head[0].copy()
+        for f in per_head[1:]:
+            best = np.maximum(best, f)
+        return best
+    raise ValueError("aggregate must be 'mean' or 'max'")
+
+
+def distance_scores(table: np.ndarray, p: int, positions: Sequence[int]) -> np.ndarray:
+    """Score of keys cached at ``positions`` for the query at p: f(p - pos)."""
+    out = np.empty(len(positions), dtype=np.float64)
+    for t, pos in enumerate(positions):
+        dist = int(p) - int(pos)
+        if dist < 0 or dist >= table.shape[0]:
+            raise ValueError(f"distance {dist} outside the table")
+        out[t] = table[dist]
+    return out
+
+
+def compress_step_distance(k_bits: np.ndarray, v_bits: np.ndarray, block_table: np.ndarray,
+                           seq_len: Sequence[int], cur_pos: Sequence[int], positions: np.ndarray,
+                           tables: np.ndarray, budget: int, window: int, sinks: int = 0,
+                           trigger: int = 0) -> Dict:
+    """``compress_step`` with distance-table scores.  positions [S][L][Hkv][>= len]
+    holds each slot's cached position; tables [L][Hkv][max_dist + 1].  The
+    returned positions are compacted with the rows."""
+    L, _, Hkv, bs, _ = k_bits.shape
+    trigger = max(int(trigger), int(budget))
+    new_k, new_v, new_pos = k_bits.copy(), v_bits.copy(), positions.copy()
+    new_len, freed = [], []
+    scores, kept_idx = {}, {}
+    for s, length in enumerate(seq_len):
+        length = int(length)
+        table_row = block_table[s]
+        if length <= trigger:
+            new_len.append(length)
+            continue
+        for l in range(L):
+            for h in range(Hkv):
+                sc = distance_scores(tables[l, h], int(cur_pos[s]), positions[s, l, h, :length])
+                idx = select(sc, length, budget, window, sinks)
+                kr = unit_rows(k_bits, table_row, length, l, h)
+                vr = unit_rows(v_bits, table_row, length, l, h)
+                store_unit_rows(new_k, table_row, compact_rows(kr, idx), l, h)
+                store_unit_rows(new_v, table_row, compact_rows(vr, idx), l, h)
+                new_pos[s, l, h, :length] = compact_rows(positions[s, l, h, :length], idx)
+                scores[(s, l, h)] = sc
+                kept_idx[(s, l, h)] = idx
+        new_len.append(budget)
+        freed += freed_blocks(table_row, length, budget, bs)
+    return {"k_pool": new_k, "v_pool": new_v, "seq_len": new_len, "freed_ids": freed,
+            "positions": new_pos, "scores": scores, "idx": kept_idx}
+
+
 def compress_step(k_vals: np.ndarray, k_bits: np.ndarray, v_bits: np.ndarray,
                   block_table: np.ndarray, seq_len: Sequence[int], cur_pos: Sequence[int],
                   qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray, G: int,

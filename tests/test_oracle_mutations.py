@@ -148,6 +148,27 @@ def _compress_step_trigger_ignored(*args, **kw):
     return _compress_step(*args, **kw)
 
 
+def _distance_series_no_conj(qbar_g, kbar, deltas, base, max_dist):
+    qb, kb = T.as_bands(np.asarray(qbar_g, np.float64)), T.as_bands(np.asarray(kbar, np.float64))
+    theta = T.rope_frequencies(qbar_g.shape[-1], base)
+    dist = np.arange(max_dist + 1, dtype=np.float64)
+    out = sum(((qb * kb)[None] * np.exp(1j * theta[None] * (dist[:, None] + d))).real.sum(-1) for d in deltas)
+    return out / len(deltas)
+
+
+def _distance_series_reversed(qbar_g, kbar, deltas, base, max_dist):
+    qb, kb = T.as_bands(np.asarray(qbar_g, np.float64)), T.as_bands(np.asarray(kbar, np.float64))
+    theta = T.rope_frequencies(qbar_g.shape[-1], base)
+    dist = np.arange(max_dist + 1, dtype=np.float64)
+    out = sum(((qb * np.conj(kb))[None] * np.exp(1j * theta[None] * (-dist[:, None] + d))).real.sum(-1)
+              for d in deltas)
+    return out / len(deltas)
+
+
+def _distance_scores_slot_not_position(table, p, positions):
+    return np.array([table[int(p) - t] for t in range(len(positions))], dtype=np.float64)
+
+
 def _compact_off_by_one(rows, idx):
     out = rows.copy()
     for j, src in enumerate(idx):
@@ -192,6 +213,9 @@ MUTATIONS = [
     ("select", _select_sinks_outside),
     ("unit_scores", _unit_scores_max_is_mean),
     ("compress_step", _compress_step_trigger_ignored),
+    ("distance_series", _distance_series_no_conj),
+    ("distance_series", _distance_series_reversed),
+    ("distance_scores", _distance_scores_slot_not_position),
     ("compact_rows", _compact_off_by_one),
     ("freed_blocks", _freed_floor),
     ("calibrate", _calibrate_vector_norms),

@@ -551,3 +551,89 @@ def test_max_over_group_matches_per_head_brute_force():
     np.testing.assert_allclose(got, per_head.max(axis=0), rtol=1e-10, atol=1e-12)
     one = oracle.unit_scores(k_post, qbar[:1], A[:1], R[:1], p, deltas, base, aggregate="max")
     np.testing.assert_allclose(one, oracle.unit_scores(k_post, qbar[:1], A[:1], R[:1], p, deltas, base), rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# Variant: the distance-only table of the centres
+# ---------------------------------------------------------------------------
+
+def test_distance_table_is_rotated_centre_logit():
+    """f(p - t) = mean_g mean_delta RoPE(qbar_g, p + delta) . RoPE(kbar, t) with
+    explicit rotation matrices, for many (p, t) with the same distance."""
+    rng = np.random.default_rng(30)
+    D, G, base = 8, 3, 1e4
+    deltas = [1, 2, 4, 9]
+    qbar = rng.normal(size=(G, D))
+    kbar = rng.normal(size=D)
+    table = oracle.distance_table(qbar, kbar, deltas, base, 60)
+    for p, t in [(50, 10), (60, 20), (45, 5), (33, 33), (60, 0), (7, 0)]:
+        want = np.mean([np.mean([_rotate_explicit(qbar[g], p + d, base) @ _rotate_explicit(kbar, t, base)
+                                 for d in deltas]) for g in range(G)])
+        assert table[p - t] == pytest.approx(want, rel=1e-11, abs=1e-12)
+    mx = oracle.distance_table(qbar, kbar, deltas, base, 60, aggregate="max")
+    per = [oracle.distance_table(qbar[g:g + 1], kbar, deltas, base, 60) for g in range(G)]
+    np.testing.assert_allclose(mx, np.max(per, axis=0), rtol=1e-14)
+
+
+def test_distance_table_equals_trig_term_of_keys_on_their_centre():
+    """Keys exactly at the key centre (k_t = RoPE(kbar, t)) with R = 1 (no
+    norm term): the method's own unit score is the table at p - t."""
+    rng = np.random.default_rng(31)
+    D, G, base, p = 16, 2, 5e5, 300
+    deltas = [1, 2, 4, 8, 16]
+    qbar = rng.normal(size=(G, D))
+    kbar = rng.normal(size=D)
+    ts = np.array([0, 1, 5, 77, 150, 299])
+    keys = np.stack([_rotate_explicit(kbar, int(t), base) for t in ts])
+    qabs = np.abs(oracle.as_bands(qbar)) + 0.5
+    got = oracle.unit_scores(keys, qbar, qabs, np.ones(G), p, deltas, base)
+    table = oracle.distance_table(qbar, kbar, deltas, base, p)
+    np.testing.assert_allclose(got, table[p - ts], rtol=1e-10, atol=1e-10)
+
+
+def test_distance_table_closed_form_two_dims():
+    """D = 2: f(dist) = |qbar||kbar| mean_delta cos(theta_0 (dist + delta) + phi)."""
+    qbar = np.array([[0.6, -1.1]])
+    kbar = np.array([1.3, 0.4])
+    deltas, base = [1, 3, 10], 1e4
+    table = oracle.distance_table(qbar, kbar, deltas, base, 40)
+    zq, zk = complex(0.6, -1.1), complex(1.3, 0.4)
+    phi = np.angle(zq) - np.angle(zk)
+    for dist in (0, 1, 17, 40):
+        want = abs(zq) * abs(zk) * np.mean([np.cos(1.0 * (dist + d) + phi) for d in deltas])
+        assert table[dist] == pytest.approx(want, rel=1e-12, abs=1e-13)
+
+
+def test_distance_step_moves_positions_with_rows():
+    """After a distance-table step the kept rows carry their positions: the
+    scores recomputed from the new positions are the kept keys' old scores,
+    and the selection is the plain selection of f(p - pos)."""
+    rng = np.random.default_rng(32)
+    L, Hkv, bs, D, S = 1, 2, 4, 8, 2
+    NB = 12
+    kb = rng.integers(-30000, 30000, size=(L, NB, Hkv, bs, D)).astype(np.int16)
+    vb = rng.integers(-30000, 30000, size=(L, NB, Hkv, bs, D)).astype(np.int16)
+    table_ids = np.array([[3, 0, 7, 5, 9, 1], [2, 4, 6, 8, 10, 11]])
+    lens, p = [21, 14], [40, 30]
+    pos = np.zeros((S, L, Hkv, 24), dtype=np.int64)
+    for s in range(S):
+        for h in range(Hkv):
+            pos[s, 0, h, :lens[s]] = np.sort(rng.choice(p[s], lens[s], replace=False))
+    tables = rng.normal(size=(L, Hkv, 41))
+    out = oracle.compress_step_distance(kb, vb, table_ids, lens, p, pos, tables, budget=8, window=2, sinks=1,
+                                        trigger=15)
+    assert out["seq_len"] == [8, 14]
+    for h in range(Hkv):
+        sc = tables[0, h, p[0] - pos[0, 0, h, :21]]
+        idx = oracle.select(sc, 21, 8, 2, 1)
+        assert np.array_equal(out["idx"][(0, 0, h)], idx)
+        assert np.array_equal(out["positions"][0, 0, h, :8], pos[0, 0, h, idx])
+        again = oracle.distance_scores(tables[0, h], p[0], out["positions"][0, 0, h, :8])
+        np.testing.assert_array_equal(again, sc[idx])
+        rows = oracle.unit_rows(out["k_pool"], table_ids[0], 8, 0, h)
+        np.testing.assert_array_equal(rows, oracle.unit_rows(kb, table_ids[0], 21, 0, h)[idx])
+    np.testing.assert_array_equal(out["positions"][1], pos[1])                 # untouched (14 <= 15)
+    assert out["freed_ids"] == [int(table_ids[0, 2]), int(table_ids[0, 3]), int(table_ids[0, 4]),
+                                int(table_ids[0, 5])]
+    with pytest.raises(ValueError):
+        oracle.distance_scores(tables[0, 0], 5, [6])                            # key after the query
