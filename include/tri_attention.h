@@ -409,6 +409,65 @@ tri_status tri_compress_step_ex(tri_kv_desc *desc, const float *qbar, const floa
 tri_status tri_reserve_blocks(const tri_kv_desc *desc, int32_t *block_table, const int32_t *n_new,
                               const tri_free_list *free_list, cudaStream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Variant: distance-only scores ([Digest] "Core Mechanism": the
+ * trigonometric series of the distance evaluated as lookups indexed by
+ * relative position; "Key Concepts", Trigonometric Distance Preference: the
+ * rotated centres' dot product depends on the query-key distance only).
+ *
+ * The key is replaced by its head's key centre kbar (the pre-rotary mean of
+ * that head's keys, e.g. tri_calibrate_centers run on key samples), so a
+ * key's score depends on its distance d = p - pos to the query alone and
+ * comes from a table built once.  The centres' norm term is the same for
+ * every key of a unit and is left out (it cannot change a ranking).
+ * ---------------------------------------------------------------------- */
+
+/*
+ * tri_distance_table - f(d) for d = 0 .. max_dist of every (layer, KV head):
+ *   f(d) = agg_g mean_delta sum_i Re( qbar_{g,i} conj(kbar_i) exp(j theta_i (d + delta)) )
+ * agg = mean (TRI_AGG_MEAN) or max (TRI_AGG_MAX) over the G query heads of
+ * the KV head.  Float64 arithmetic, stored fp32.
+ *   L, Hkv, G, D : shapes (Hq = Hkv*G; D must be 128)
+ *   qbar   : f32 [L][Hq][D] query centres;  kbar : f32 [L][Hkv][D] key centres
+ *   deltas : HOST int32 [n_deltas], 1 <= n_deltas <= TRI_MAX_DELTAS
+ *   max_dist : 1 <= max_dist < 2^24
+ *   table  : f32 [L][Hkv][max_dist + 1] out
+ * Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED (D != 128; TRI_AGG_MAX with
+ * G > 64), TRI_ERR_CUDA.
+ */
+tri_status tri_distance_table(int L, int Hkv, int G, int D, const float *qbar, const float *kbar,
+                              double rope_base, const int32_t *deltas, int n_deltas, int aggregate,
+                              int max_dist, float *table, cudaStream_t stream);
+
+/*
+ * tri_score_distance - scores[s][l][h][t] = table[l][h][cur_pos[s] - pos] with
+ * pos = slot_pos[s][l][h][t], for t < seq_len[s]; the rest is not written.
+ *   slot_pos : int32 [S][L][Hkv][max_blocks*16], the position each slot's key
+ *              was cached at (slot_pos[...][t] = t for a cache never compacted)
+ *   table, max_dist : as built by tri_distance_table for this cache's L, Hkv
+ *   scores   : f32 [S][L][Hkv][max_blocks*16]
+ * A distance outside [0, max_dist] raises TRI_DEVFLAG_BOUNDS (the nearest
+ * table entry is used).  Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED,
+ * TRI_ERR_CUDA.
+ */
+tri_status tri_score_distance(const tri_kv_desc *desc, const float *table, int max_dist,
+                              const int32_t *slot_pos, float *scores, cudaStream_t stream);
+
+/*
+ * tri_compress_step_distance - tri_compress_step_ex with the table's scores:
+ * no pass over the cached keys.  slot_pos (layout as above) is compacted with
+ * the rows: slot j of a compressed unit takes the position of old slot
+ * idx[j].  opt->aggregate is ignored (the table fixes it).
+ *   workspace : >= tri_workspace_size(desc, opt->budget) bytes.
+ * Other arguments, results, errors and flags: as tri_compress_step_ex.
+ */
+tri_status tri_compress_step_distance(tri_kv_desc *desc, const float *table, int max_dist,
+                                      int32_t *slot_pos, const tri_step_options *opt,
+                                      const tri_free_list *free_list, int32_t *freed_ids,
+                                      int32_t *freed_count, int32_t *idx_out, void *workspace,
+                                      size_t ws_bytes, const tri_phase_events *events,
+                                      cudaStream_t stream);
+
 /*
  * tri_sync_status - wait for `stream`, read the device status word, clear it,
  * and return TRI_OK or the error its bits name (BOUNDS before TIMEOUT before

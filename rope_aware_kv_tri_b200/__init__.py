@@ -43,7 +43,8 @@ EXPORTS = (
     "tri_calibrate_centers", "tri_build_query", "tri_workspace_size", "tri_score",
     "tri_select_topk", "tri_compact_kv", "tri_compress_step", "tri_compress_step_static_scratch",
     "tri_sync_status", "tri_status_string", "tri_workspace_size_ex", "tri_score_ex", "tri_select_topk_ex",
-    "tri_compress_step_ex", "tri_reserve_blocks",
+    "tri_compress_step_ex", "tri_reserve_blocks", "tri_distance_table", "tri_score_distance",
+    "tri_compress_step_distance",
 )
 TRI_STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -151,6 +152,11 @@ def _load() -> ctypes.CDLL:
                                      ctypes.POINTER(TriFreeList), P, P, P, P, S,
                                      ctypes.POINTER(TriPhaseEvents), P]),
         "tri_reserve_blocks": (I, [desc_p, P, P, ctypes.POINTER(TriFreeList), P]),
+        "tri_distance_table": (I, [I, I, I, I, P, P, D, P, I, I, I, P, P]),
+        "tri_score_distance": (I, [desc_p, P, I, P, P, P]),
+        "tri_compress_step_distance": (I, [desc_p, P, I, P, ctypes.POINTER(TriStepOptions),
+                                           ctypes.POINTER(TriFreeList), P, P, P, P, S,
+                                           ctypes.POINTER(TriPhaseEvents), P]),
         "tri_status_string": (ctypes.c_char_p, [I]),
     }
     for name, (res, args) in sig.items():
@@ -370,6 +376,40 @@ def tri_reserve_blocks(cache: KvCache, n_new, free_list: FreeList, stream=None) 
         cache.ref, _ptr(cache.tensors[2], torch.int32, "block_table"), _ptr(n_new, torch.int32, "n_new"),
         free_list.ref, _stream(stream))
     _check(code, "tri_reserve_blocks")
+
+
+def tri_distance_table(qbar, kbar, rope_base: float, deltas, aggregate: int, table, stream=None) -> None:
+    """qbar f32 [L][Hq][D], kbar f32 [L][Hkv][D] -> table f32 [L][Hkv][max_dist + 1]."""
+    L, Hq, D = qbar.shape
+    Hkv = kbar.shape[1]
+    if Hq % Hkv or tuple(kbar.shape) != (L, Hkv, D) or table.dim() != 3 or tuple(table.shape[:2]) != (L, Hkv):
+        raise ValueError("inconsistent shapes")
+    arr, n = _deltas(deltas)
+    code = library().tri_distance_table(
+        L, Hkv, Hq // Hkv, D, _ptr(qbar, torch.float32, "qbar"), _ptr(kbar, torch.float32, "kbar"),
+        float(rope_base), arr, n, int(aggregate), table.shape[2] - 1, _ptr(table, torch.float32, "table"),
+        _stream(stream))
+    _check(code, "tri_distance_table")
+
+
+def tri_score_distance(cache: KvCache, table, slot_pos, scores, stream=None) -> None:
+    code = library().tri_score_distance(
+        cache.ref, _ptr(table, torch.float32, "table"), table.shape[-1] - 1, _ptr(slot_pos, torch.int32, "slot_pos"),
+        _ptr(scores, torch.float32, "scores"), _stream(stream))
+    _check(code, "tri_score_distance")
+
+
+def tri_compress_step_distance(cache: KvCache, table, slot_pos, opt: TriStepOptions, workspace,
+                               free_list: Optional[FreeList] = None, freed_ids=None, freed_count=None,
+                               idx_out=None, events=None, stream=None) -> None:
+    code = library().tri_compress_step_distance(
+        cache.ref, _ptr(table, torch.float32, "table"), table.shape[-1] - 1, _ptr(slot_pos, torch.int32, "slot_pos"),
+        ctypes.byref(opt), free_list.ref if free_list is not None else None,
+        _ptr(freed_ids, torch.int32, "freed_ids", allow_none=True),
+        _ptr(freed_count, torch.int32, "freed_count", allow_none=True),
+        _ptr(idx_out, torch.int32, "idx_out", allow_none=True),
+        _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _events(events), _stream(stream))
+    _check(code, "tri_compress_step_distance")
 
 
 def tri_sync_status(status, stream=None) -> int:

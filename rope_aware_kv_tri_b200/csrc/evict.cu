@@ -113,6 +113,8 @@ struct EvictSmem {
     int n_list;
 };
 
+static_assert(sizeof(SelectScratch) >= TRI_MAX_BUDGET * sizeof(int), "position staging does not fit");
+
 // rows per ordered compaction round, staged in the selection scratch
 constexpr int kStageRows = (int)(sizeof(SelectScratch) / (2 * kRowBytes));
 
@@ -897,6 +899,16 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
         }
     }
     if (p.do_compact) {
+        if (p.slot_pos) {
+            // Positions travel with their rows: every kept position is read
+            // into the (now idle) selection scratch before any is stored.
+            int32_t* pos = p.slot_pos + (int64_t)u * p.pos_stride;
+            int* stage = reinterpret_cast<int*>(&sm.u);
+            for (int j = threadIdx.x; j < kept; j += kEvictThreads) stage[j] = pos[sidx[j]];
+            __syncthreads();
+            for (int j = threadIdx.x; j < kept; j += kEvictThreads) pos[j] = stage[j];
+            __syncthreads();
+        }
         int fixed = 0, low = 0;
         for (int j = threadIdx.x; j < kept; j += kEvictThreads) {
             fixed += (sidx[j] == j) ? 1 : 0;

@@ -134,6 +134,13 @@ __device__ void plan_sequences(const QueryParams& p) {
         carry_items += tot_i;
         carry_freed += tot_f;
     }
+    if (p.plan_only && p.unit_kmin) {
+        const int U = p.S * p.L * p.Hkv;
+        for (int u = threadIdx.x; u < U; u += kQueryThreads) {
+            p.unit_kmin[u] = 0xffffffffu;
+            p.unit_kmax[u] = 0u;
+        }
+    }
     if (threadIdx.x == 0) {
         p.item_off[p.S] = carry_items;
         p.freed_off[p.S] = carry_freed;
@@ -167,6 +174,10 @@ __global__ void __launch_bounds__(kQueryThreads) query_kernel(const QueryParams 
 }  // namespace
 
 cudaError_t launch_query(const QueryParams& p, cudaStream_t stream) {
+    if (p.plan_only) {
+        query_kernel<<<1, kQueryThreads, 0, stream>>>(p, 0);
+        return cudaGetLastError();
+    }
     const int per_seq = (p.L * p.Hkv + kUnitsPerCta - 1) / kUnitsPerCta;
     query_kernel<<<p.S * per_seq + (p.do_plan ? 1 : 0), kQueryThreads, 0, stream>>>(p, per_seq);
     return cudaGetLastError();

@@ -25,7 +25,8 @@
 //    quarter of one), so its 24 coefficients stay in registers for the whole
 //    item.  8 lanes share a key: lane `sub` reads 16 bytes of the real half
 //    (dims 8sub..8sub+7) and the matching 16 bytes of the imaginary half
-//    (dims 64+8sub..), i.e. 8 whole bands; fp32 FMA; 3 xor-shuffles reduce.
+//    (dims 64+8sub..), i.e. 8 whole bands; fp32 FMA on packed pairs of
+//    adjacent bands (fma.rn.f32x2); 3 xor-shuffles reduce.
 //  * Each warp also tracks the smallest and largest order key of the scores
 //    it writes for a unit and folds them into the unit's key range with one
 //    atomicMin/atomicMax per item; the selection buckets scores linearly over
@@ -73,23 +74,23 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     return false;
 }
 
-__device__ __forceinline__ float key_score(const uint4 a, const uint4 b, const float (&qr)[8],
-                                           const float (&qi)[8], const float (&ww)[8]) {
+// This lane's part of a key score: 8 bands (4 adjacent pairs) of the real
+// half a and the imaginary half b, with packed-pair fp32 arithmetic.
+__device__ __forceinline__ float key_score(const uint4 a, const uint4 b, const float2 (&qr)[4],
+                                           const float2 (&qi)[4], const float2 (&ww)[4]) {
     const uint32_t av[4] = {a.x, a.y, a.z, a.w};
     const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
-    float dot0 = 0.f, dot1 = 0.f, nrm0 = 0.f, nrm1 = 0.f;
+    float2 dot = make_float2(0.f, 0.f), nrm = make_float2(0.f, 0.f);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const float r0 = bf16_lo(av[j]), r1 = bf16_hi(av[j]);
-        const float i0 = bf16_lo(bv[j]), i1 = bf16_hi(bv[j]);
-        dot0 = fmaf(qr[2 * j], r0, dot0);
-        dot1 = fmaf(qr[2 * j + 1], r1, dot1);
-        dot0 = fmaf(qi[2 * j], i0, dot0);
-        dot1 = fmaf(qi[2 * j + 1], i1, dot1);
-        nrm0 = fmaf(ww[2 * j], sqrt_fast(fmaf(r0, r0, i0 * i0)), nrm0);
-        nrm1 = fmaf(ww[2 * j + 1], sqrt_fast(fmaf(r1, r1, i1 * i1)), nrm1);
+        const float2 r = make_float2(bf16_lo(av[j]), bf16_hi(av[j]));
+        const float2 i = make_float2(bf16_lo(bv[j]), bf16_hi(bv[j]));
+        dot = ffma2(qr[j], r, dot);
+        dot = ffma2(qi[j], i, dot);
+        const float2 sq = ffma2(r, r, fmul2(i, i));
+        nrm = ffma2(ww[j], make_float2(sqrt_fast(sq.x), sqrt_fast(sq.y)), nrm);
     }
-    return (dot0 + dot1) + (nrm0 + nrm1);
+    return (dot.x + dot.y) + (nrm.x + nrm.y);
 }
 
 // ---- max over the group -------------------------------------------------
@@ -101,9 +102,11 @@ template <> struct MaxLayout<4> { static constexpr int kBpl = 4; };
 template <> struct MaxLayout<8> { static constexpr int kBpl = 2; };
 
 // BPL bf16 values of the real half (dims sub*BPL..) and of the imaginary
-// half (dims 64 + sub*BPL..) of a 256-byte key row.
+// half (dims 64 + sub*BPL..) of a 256-byte key row, as pairs of adjacent
+// bands (element j of a pair array holds bands 2j and 2j+1 of the lane).
 template <int BPL>
-__device__ __forceinline__ void load_bands(const uint8_t* row, int sub, float (&re)[BPL], float (&im)[BPL]) {
+__device__ __forceinline__ void load_bands(const uint8_t* row, int sub, float2 (&re)[BPL / 2],
+                                           float2 (&im)[BPL / 2]) {
     constexpr int W = BPL / 2;                 // 32-bit words per half
     uint32_t a[W], b[W];
     if constexpr (W == 4) {
@@ -122,10 +125,8 @@ __device__ __forceinline__ void load_bands(const uint8_t* row, int sub, float (&
     }
 #pragma unroll
     for (int j = 0; j < W; ++j) {
-        re[2 * j] = bf16_lo(a[j]);
-        re[2 * j + 1] = bf16_hi(a[j]);
-        im[2 * j] = bf16_lo(b[j]);
-        im[2 * j + 1] = bf16_hi(b[j]);
+        re[j] = make_float2(bf16_lo(a[j]), bf16_hi(a[j]));
+        im[j] = make_float2(bf16_lo(b[j]), bf16_hi(b[j]));
     }
 }
 
@@ -251,7 +252,7 @@ __device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t*
     const int hig = warp / wph;                // head of the tile group
     const int q0 = warp % wph;                 // first quad of keys
     const int sub = lane & 7, kq = lane >> 3;
-    float qr[8], qi[8], ww[8];
+    float2 qr[4], qi[4], ww[4];
     int cur_unit = -1;
     const uint64_t keep_pol = l2_policy_evict_last();   // scores are re-read by the selection
     // order-key range of the scores this warp wrote for cur_unit
@@ -287,12 +288,12 @@ __device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t*
                 const float4 x0 = qe[2 * sub], x1 = qe[2 * sub + 1];
                 const float4 y0 = qe[16 + 2 * sub], y1 = qe[16 + 2 * sub + 1];
                 const float4 z0 = we[2 * sub], z1 = we[2 * sub + 1];
-                qr[0] = x0.x; qr[1] = x0.y; qr[2] = x0.z; qr[3] = x0.w;
-                qr[4] = x1.x; qr[5] = x1.y; qr[6] = x1.z; qr[7] = x1.w;
-                qi[0] = y0.x; qi[1] = y0.y; qi[2] = y0.z; qi[3] = y0.w;
-                qi[4] = y1.x; qi[5] = y1.y; qi[6] = y1.z; qi[7] = y1.w;
-                ww[0] = z0.x; ww[1] = z0.y; ww[2] = z0.z; ww[3] = z0.w;
-                ww[4] = z1.x; ww[5] = z1.y; ww[6] = z1.z; ww[7] = z1.w;
+                qr[0] = make_float2(x0.x, x0.y); qr[1] = make_float2(x0.z, x0.w);
+                qr[2] = make_float2(x1.x, x1.y); qr[3] = make_float2(x1.z, x1.w);
+                qi[0] = make_float2(y0.x, y0.y); qi[1] = make_float2(y0.z, y0.w);
+                qi[2] = make_float2(y1.x, y1.y); qi[3] = make_float2(y1.z, y1.w);
+                ww[0] = make_float2(z0.x, z0.y); ww[1] = make_float2(z0.z, z0.w);
+                ww[2] = make_float2(z1.x, z1.y); ww[3] = make_float2(z1.z, z1.w);
                 cur_unit = unit;
             }
             const uint8_t* tile = tiles + (size_t)slot * stage_bytes + (size_t)hig * kTileBytes;
@@ -330,8 +331,9 @@ __device__ void consume_max(const ScoreParams& p, int warp, int lane, const uint
     const int wph = kConsumerWarps / HG;
     const int hig = warp / wph;
     const int q0 = warp % wph;
+    constexpr int NP = BPL / 2;                // band pairs per lane
     const int sub = lane % LPK, kq = lane / LPK;
-    float qr[G][BPL], qi[G][BPL], ww[G][BPL];
+    float2 qr[G][NP], qi[G][NP], ww[G][NP];
     int cur_unit = -1;
     const uint64_t keep_pol = l2_policy_evict_last();
     uint32_t kmin = 0xffffffffu, kmax = 0u;
@@ -363,13 +365,13 @@ __device__ void consume_max(const ScoreParams& p, int warp, int lane, const uint
                 flush_range();
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    const float* qe = p.qeff + ((int64_t)unit * G + g) * kHeadDim;
-                    const float* we = p.wts + ((int64_t)unit * G + g) * kBands;
+                    const float2* qe = reinterpret_cast<const float2*>(p.qeff + ((int64_t)unit * G + g) * kHeadDim);
+                    const float2* we = reinterpret_cast<const float2*>(p.wts + ((int64_t)unit * G + g) * kBands);
 #pragma unroll
-                    for (int b = 0; b < BPL; ++b) {
-                        qr[g][b] = __ldg(qe + sub * BPL + b);
-                        qi[g][b] = __ldg(qe + kBands + sub * BPL + b);
-                        ww[g][b] = __ldg(we + sub * BPL + b);
+                    for (int j = 0; j < NP; ++j) {
+                        qr[g][j] = __ldg(qe + sub * NP + j);
+                        qi[g][j] = __ldg(qe + kBands / 2 + sub * NP + j);
+                        ww[g][j] = __ldg(we + sub * NP + j);
                     }
                 }
                 cur_unit = unit;
@@ -378,21 +380,24 @@ __device__ void consume_max(const ScoreParams& p, int warp, int lane, const uint
             float* out = p.scores + (int64_t)unit * p.score_stride + m.t0;
             for (int q = q0; q < kBlockRows / KPI; q += wph) {
                 const int row = q * KPI + kq;
-                float re[BPL], im[BPL], nrm[BPL];
+                float2 re[NP], im[NP], nrm[NP];
                 load_bands<BPL>(tile + row * 256, sub, re, im);
 #pragma unroll
-                for (int b = 0; b < BPL; ++b) nrm[b] = sqrt_fast(fmaf(re[b], re[b], im[b] * im[b]));
+                for (int j = 0; j < NP; ++j) {
+                    const float2 sq = ffma2(re[j], re[j], fmul2(im[j], im[j]));
+                    nrm[j] = make_float2(sqrt_fast(sq.x), sqrt_fast(sq.y));
+                }
                 float v[G];
 #pragma unroll
                 for (int g = 0; g < G; ++g) {
-                    float d0 = 0.f, d1 = 0.f;
+                    float2 d0 = make_float2(0.f, 0.f), d1 = make_float2(0.f, 0.f);
 #pragma unroll
-                    for (int b = 0; b < BPL; ++b) {
-                        d0 = fmaf(qr[g][b], re[b], d0);
-                        d1 = fmaf(qi[g][b], im[b], d1);
-                        d0 = fmaf(ww[g][b], nrm[b], d0);
+                    for (int j = 0; j < NP; ++j) {
+                        d0 = ffma2(qr[g][j], re[j], d0);
+                        d1 = ffma2(qi[g][j], im[j], d1);
+                        d0 = ffma2(ww[g][j], nrm[j], d0);
                     }
-                    v[g] = d0 + d1;
+                    v[g] = (d0.x + d0.y) + (d1.x + d1.y);
                 }
                 const float acc = group_max<G, LPK>(v, lane);
                 if (sub == 0 && row < m.nrows) {

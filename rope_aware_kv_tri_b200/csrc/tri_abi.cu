@@ -235,6 +235,92 @@ void record(cudaEvent_t ev, cudaStream_t stream) {
     if (ev) cudaEventRecord(ev, stream);
 }
 
+// The selection and compaction launches of a step, after its scores are in
+// the workspace (evict: select + plan + at-risk rows; copy-out; move).
+tri_status select_and_compact(const tri_kv_desc* desc, uint8_t* ws, const WsLayout& w, const tri_step_options& opt,
+                              int trigger, const tri_free_list* free_list, int32_t* freed_ids, int32_t* idx_out,
+                              int32_t* slot_pos, bool pdl, cudaStream_t stream) {
+    const int budget = opt.budget;
+    EvictParams e = make_evict_params(desc);
+    e.scores = reinterpret_cast<const float*>(ws + w.scores);
+    e.unit_kmin = reinterpret_cast<const uint32_t*>(ws + w.kmin);
+    e.unit_kmax = reinterpret_cast<const uint32_t*>(ws + w.kmax);
+    e.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
+    e.budget = budget;
+    e.window = opt.window;
+    e.sinks = opt.sinks;
+    e.trigger = trigger;
+    e.idx_out = reinterpret_cast<int32_t*>(ws + w.idx);
+    e.idx_copy = idx_out;
+    e.do_select = 1;
+    e.do_compact = 1;
+    e.seq_len_out = desc->seq_len;
+    e.freed_off = reinterpret_cast<const int32_t*>(ws + w.freed_off);
+    e.freed_ids = freed_ids;
+    if (free_list) {
+        e.fl_ids = free_list->ids;
+        e.fl_base = reinterpret_cast<const int32_t*>(ws + w.words) + 2;
+    }
+    e.slot_pos = slot_pos;
+    e.pos_stride = (int64_t)desc->max_blocks * kBlockRows;
+    e.scratch_used = reinterpret_cast<int32_t*>(ws + w.words);
+    e.unit_info = reinterpret_cast<int32_t*>(ws + w.info);
+    e.scratch_owner = reinterpret_cast<int32_t*>(ws + w.owner);
+    e.scratch_rows = w.scratch_rows;
+    tri_status st;
+    if ((st = cuda_status(launch_evict(e, stream, pdl))) != TRI_OK) return st;
+    MoveParams mv = make_move_params(desc, reinterpret_cast<const int32_t*>(ws + w.idx), budget);
+    mv.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
+    mv.kept = nullptr;
+    mv.trigger = trigger;
+    mv.unit_info = reinterpret_cast<const int32_t*>(ws + w.info);
+    mv.scratch = ws + w.scratch;
+    mv.scratch_owner = reinterpret_cast<const int32_t*>(ws + w.owner);
+    mv.scratch_used = reinterpret_cast<const int32_t*>(ws + w.words);
+    mv.scratch_rows = w.scratch_rows;
+    mv.copy_out = 1;
+    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream, pdl))) != TRI_OK) return st;
+    mv.copy_out = 0;
+    return cuda_status(launch_move(mv, device_sm_count(), stream, pdl));
+}
+
+// Step outputs: freed ids + count (both or neither), a free list, idx.
+tri_status check_step_outputs(const tri_free_list* free_list, const int32_t* freed_ids, const int32_t* freed_count,
+                              const int32_t* idx_out) {
+    tri_status st = check_free_list(free_list);
+    if (st != TRI_OK) return st;
+    if ((freed_ids == nullptr) != (freed_count == nullptr)) return TRI_ERR_INVALID;
+    if (!freed_ids && !free_list) return TRI_ERR_INVALID;
+    if ((freed_ids && !aligned(freed_ids, 4)) || (freed_count && !aligned(freed_count, 4))) return TRI_ERR_INVALID;
+    if (idx_out && !aligned(idx_out, 4)) return TRI_ERR_INVALID;
+    return TRI_OK;
+}
+
+DistScoreParams make_distance_params(const tri_kv_desc* desc, const float* table, int max_dist,
+                                     const int32_t* slot_pos, float* scores) {
+    DistScoreParams d{};
+    d.table = table;
+    d.max_dist = max_dist;
+    d.slot_pos = slot_pos;
+    d.pos_stride = (int64_t)desc->max_blocks * kBlockRows;
+    d.cur_pos = desc->cur_pos;
+    d.lens = desc->seq_len;
+    d.trigger = -1;
+    d.scores = scores;
+    d.score_stride = (int64_t)desc->max_blocks * kBlockRows;
+    d.L = desc->L;
+    d.Hkv = desc->Hkv;
+    d.S = desc->S;
+    d.status = desc->status;
+    return d;
+}
+
+tri_status check_distance_args(const float* table, int max_dist, const int32_t* slot_pos) {
+    if (!table || !slot_pos || !aligned(table, 4) || !aligned(slot_pos, 4)) return TRI_ERR_INVALID;
+    if (max_dist < 1 || max_dist >= (1 << 24)) return TRI_ERR_INVALID;
+    return TRI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -394,11 +480,7 @@ tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const floa
     if ((st = check_stats(qbar, qabs, R)) != TRI_OK) return st;
     if ((st = check_query_args(rope_base, deltas, n_deltas)) != TRI_OK) return st;
     if ((st = check_options(opt, desc->G)) != TRI_OK) return st;
-    if ((st = check_free_list(free_list)) != TRI_OK) return st;
-    if ((freed_ids == nullptr) != (freed_count == nullptr)) return TRI_ERR_INVALID;
-    if (!freed_ids && !free_list) return TRI_ERR_INVALID;
-    if ((freed_ids && !aligned(freed_ids, 4)) || (freed_count && !aligned(freed_count, 4))) return TRI_ERR_INVALID;
-    if (idx_out && !aligned(idx_out, 4)) return TRI_ERR_INVALID;
+    if ((st = check_step_outputs(free_list, freed_ids, freed_count, idx_out)) != TRI_OK) return st;
     const int budget = opt->budget;
     const bool per_head = opt->aggregate == TRI_AGG_MAX;
     if ((st = check_workspace(desc, workspace, ws_bytes, budget, per_head)) != TRI_OK) return st;
@@ -446,44 +528,112 @@ tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const floa
         return st;
     if (events) record(events->after_score, stream);
 
-    EvictParams e = make_evict_params(desc);
-    e.scores = scores;
-    e.unit_kmin = reinterpret_cast<const uint32_t*>(ws + w.kmin);
-    e.unit_kmax = reinterpret_cast<const uint32_t*>(ws + w.kmax);
-    e.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
-    e.budget = budget;
-    e.window = opt->window;
-    e.sinks = opt->sinks;
-    e.trigger = trigger;
-    e.idx_out = reinterpret_cast<int32_t*>(ws + w.idx);
-    e.idx_copy = idx_out;
-    e.do_select = 1;
-    e.do_compact = 1;
-    e.seq_len_out = desc->seq_len;
-    e.freed_off = reinterpret_cast<const int32_t*>(ws + w.freed_off);
-    e.freed_ids = freed_ids;
-    if (free_list) {
-        e.fl_ids = free_list->ids;
-        e.fl_base = reinterpret_cast<const int32_t*>(ws + w.words) + 2;
+    if ((st = select_and_compact(desc, ws, w, *opt, trigger, free_list, freed_ids, idx_out, nullptr, pdl, stream)) !=
+        TRI_OK)
+        return st;
+    if (events) record(events->after_evict, stream);
+    return TRI_OK;
+}
+
+tri_status tri_distance_table(int L, int Hkv, int G, int D, const float* qbar, const float* kbar, double rope_base,
+                              const int32_t* deltas, int n_deltas, int aggregate, int max_dist, float* table,
+                              cudaStream_t stream) {
+    if (L < 1 || Hkv < 1 || G < 1 || (int64_t)L * Hkv > INT_MAX || (int64_t)Hkv * G > INT_MAX) return TRI_ERR_INVALID;
+    if (D != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
+    if (!qbar || !kbar || !table || !aligned(qbar, 4) || !aligned(kbar, 4) || !aligned(table, 4))
+        return TRI_ERR_INVALID;
+    tri_status st = check_query_args(rope_base, deltas, n_deltas);
+    if (st != TRI_OK) return st;
+    if (aggregate != TRI_AGG_MEAN && aggregate != TRI_AGG_MAX) return TRI_ERR_INVALID;
+    if (aggregate == TRI_AGG_MAX && G > 64) return TRI_ERR_UNSUPPORTED;
+    if (max_dist < 1 || max_dist >= (1 << 24)) return TRI_ERR_INVALID;
+    DistTableParams t{};
+    t.qbar = qbar;
+    t.kbar = kbar;
+    t.base = rope_base;
+    t.n_deltas = n_deltas;
+    for (int i = 0; i < n_deltas; ++i) t.deltas[i] = deltas[i];
+    t.L = L;
+    t.Hkv = Hkv;
+    t.G = G;
+    t.per_head = aggregate == TRI_AGG_MAX ? 1 : 0;
+    t.max_dist = max_dist;
+    t.table = table;
+    return cuda_status(launch_distance_table(t, stream));
+}
+
+tri_status tri_score_distance(const tri_kv_desc* desc, const float* table, int max_dist, const int32_t* slot_pos,
+                              float* scores, cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if ((st = check_distance_args(table, max_dist, slot_pos)) != TRI_OK) return st;
+    if (!scores || !aligned(scores, 4)) return TRI_ERR_INVALID;
+    if (desc->S == 0) return TRI_OK;
+    return cuda_status(launch_distance_score(make_distance_params(desc, table, max_dist, slot_pos, scores), stream));
+}
+
+tri_status tri_compress_step_distance(tri_kv_desc* desc, const float* table, int max_dist, int32_t* slot_pos,
+                                      const tri_step_options* opt, const tri_free_list* free_list, int32_t* freed_ids,
+                                      int32_t* freed_count, int32_t* idx_out, void* workspace, size_t ws_bytes,
+                                      const tri_phase_events* events, cudaStream_t stream) {
+    tri_status st = check_desc(desc);
+    if (st != TRI_OK) return st;
+    if ((st = check_distance_args(table, max_dist, slot_pos)) != TRI_OK) return st;
+    if ((st = check_options(opt, 0)) != TRI_OK) return st;
+    if ((st = check_step_outputs(free_list, freed_ids, freed_count, idx_out)) != TRI_OK) return st;
+    const int budget = opt->budget;
+    if ((st = check_workspace(desc, workspace, ws_bytes, budget)) != TRI_OK) return st;
+    if (events) record(events->start, stream);
+    if (desc->S == 0) {
+        st = freed_count ? cuda_status(cudaMemsetAsync(freed_count, 0, sizeof(int32_t), stream)) : TRI_OK;
+        if (events) {
+            record(events->after_query, stream);
+            record(events->after_score, stream);
+            record(events->after_evict, stream);
+        }
+        return st;
     }
-    e.scratch_used = reinterpret_cast<int32_t*>(ws + w.words);
-    e.unit_info = reinterpret_cast<int32_t*>(ws + w.info);
-    e.scratch_owner = reinterpret_cast<int32_t*>(ws + w.owner);
-    e.scratch_rows = w.scratch_rows;
-    if ((st = cuda_status(launch_evict(e, stream, pdl))) != TRI_OK) return st;
-    MoveParams mv = make_move_params(desc, reinterpret_cast<const int32_t*>(ws + w.idx), budget);
-    mv.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
-    mv.kept = nullptr;
-    mv.trigger = trigger;
-    mv.unit_info = reinterpret_cast<const int32_t*>(ws + w.info);
-    mv.scratch = ws + w.scratch;
-    mv.scratch_owner = reinterpret_cast<const int32_t*>(ws + w.owner);
-    mv.scratch_used = reinterpret_cast<const int32_t*>(ws + w.words);
-    mv.scratch_rows = w.scratch_rows;
-    mv.copy_out = 1;
-    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream, pdl))) != TRI_OK) return st;
-    mv.copy_out = 0;
-    if ((st = cuda_status(launch_move(mv, device_sm_count(), stream, pdl))) != TRI_OK) return st;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const WsLayout w = ws_layout(desc, budget);
+    const int trigger = effective_trigger(*opt);
+    QueryParams q{};
+    q.L = desc->L;
+    q.Hkv = desc->Hkv;
+    q.G = desc->G;
+    q.S = desc->S;
+    q.seq_len = desc->seq_len;
+    q.max_blocks = desc->max_blocks;
+    q.heads_per_tile = score_heads_per_tile(desc->Hkv);
+    q.status = desc->status;
+    q.plan_only = 1;
+    q.do_plan = 1;
+    q.budget = budget;
+    q.trigger = trigger;
+    q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
+    q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
+    q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
+    q.freed_count = freed_count;
+    q.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
+    q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
+    q.zero_words = reinterpret_cast<int32_t*>(ws + w.words);
+    if (free_list) {
+        q.fl_count = free_list->count;
+        q.fl_capacity = free_list->capacity;
+        q.fl_base = reinterpret_cast<int32_t*>(ws + w.words) + 2;
+    }
+    if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
+    if (events) record(events->after_query, stream);
+    const bool pdl = events == nullptr;
+    DistScoreParams d = make_distance_params(desc, table, max_dist, slot_pos, reinterpret_cast<float*>(ws + w.scores));
+    d.lens = reinterpret_cast<const int32_t*>(ws + w.len_ws);
+    d.trigger = trigger;
+    d.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
+    d.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
+    if ((st = cuda_status(launch_distance_score(d, stream, pdl))) != TRI_OK) return st;
+    if (events) record(events->after_score, stream);
+    if ((st = select_and_compact(desc, ws, w, *opt, trigger, free_list, freed_ids, idx_out, slot_pos, pdl, stream)) !=
+        TRI_OK)
+        return st;
     if (events) record(events->after_evict, stream);
     return TRI_OK;
 }

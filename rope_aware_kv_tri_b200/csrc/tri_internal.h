@@ -61,6 +61,7 @@ struct QueryParams {
     uint32_t* unit_kmin;      // [U] set to the largest key (min accumulator) or null
     uint32_t* unit_kmax;      // [U] set to 0 (max accumulator) or null
     int32_t* zero_words;      // [2] set to 0 by the plan CTA, or null
+    int plan_only;            // 1: the plan CTA alone (no effective queries)
     int32_t* fl_count;        // free list to push the freed ids on, or null
     int fl_capacity;
     int32_t* fl_base;         // [1] out: first list entry of this step's ids, -1 if no room
@@ -115,6 +116,8 @@ struct EvictParams {
     int32_t* freed_ids;        // or null
     int32_t* fl_ids;           // free list entries, or null
     const int32_t* fl_base;    // [1] where this step's ids start in fl_ids (-1: none)
+    int32_t* slot_pos;         // [U][pos_stride] cached position of every slot, compacted with the rows, or null
+    int64_t pos_stride;
     int32_t* status;
     // step plans (null outside tri_compress_step)
     int32_t* scratch_used;     // [1] rows of the scratch handed out, 0 at launch
@@ -156,6 +159,37 @@ struct FinalizeParams {
     int32_t* status;
 };
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t stream);
+
+// ------------------------------------------------------ distance variant
+struct DistTableParams {
+    const float* qbar;        // [L][Hq][D]
+    const float* kbar;        // [L][Hkv][D]
+    double base;
+    int n_deltas;
+    int32_t deltas[TRI_MAX_DELTAS];
+    int L, Hkv, G;
+    int per_head;             // 1: max over the group, 0: mean (folded)
+    int max_dist;
+    float* table;             // [L][Hkv][max_dist + 1]
+};
+cudaError_t launch_distance_table(const DistTableParams& p, cudaStream_t stream);
+
+struct DistScoreParams {
+    const float* table;
+    int max_dist;
+    const int32_t* slot_pos;  // [U][pos_stride]
+    int64_t pos_stride;       // max_blocks * 16
+    const int64_t* cur_pos;
+    const int32_t* lens;      // [S]
+    int trigger;              // units of sequences with len <= trigger are skipped (-1: none)
+    float* scores;
+    int64_t score_stride;
+    uint32_t* unit_kmin;      // [U] or null (initialised by the plan)
+    uint32_t* unit_kmax;
+    int L, Hkv, S;
+    int32_t* status;
+};
+cudaError_t launch_distance_score(const DistScoreParams& p, cudaStream_t stream, bool pdl = false);
 
 // Pop blocks for n_new[s] more slots per sequence from a device free list.
 struct ReserveParams {

@@ -219,3 +219,33 @@ def test_reserve_rejects(lib):
     assert lib.tri_reserve_blocks(ctypes.byref(d), FAKE, None, ctypes.byref(fl), None) == tri.TRI_ERR_INVALID
     assert lib.tri_reserve_blocks(ctypes.byref(_desc(D=64)), FAKE, FAKE, ctypes.byref(fl),
                                   None) == tri.TRI_ERR_UNSUPPORTED
+
+
+def test_distance_entries_reject(lib):
+    arr = (ctypes.c_int32 * 2)(1, 2)
+    ok = dict(L=2, Hkv=8, G=4, D=128, qbar=FAKE, kbar=FAKE, base=1e4, deltas=arr, n=2, agg=0, max_dist=100, table=FAKE)
+
+    def table(**kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.tri_distance_table(a["L"], a["Hkv"], a["G"], a["D"], a["qbar"], a["kbar"], a["base"],
+                                      a["deltas"], a["n"], a["agg"], a["max_dist"], a["table"], None)
+    assert table(D=64) == tri.TRI_ERR_UNSUPPORTED
+    assert table(L=0) == tri.TRI_ERR_INVALID
+    assert table(kbar=None) == tri.TRI_ERR_INVALID
+    assert table(max_dist=0) == tri.TRI_ERR_INVALID
+    assert table(max_dist=1 << 24) == tri.TRI_ERR_INVALID
+    assert table(agg=9) == tri.TRI_ERR_INVALID
+    assert table(agg=tri.TRI_AGG_MAX, G=65) == tri.TRI_ERR_UNSUPPORTED
+    assert table(n=0) == tri.TRI_ERR_INVALID
+    d = _desc()
+    assert lib.tri_score_distance(ctypes.byref(d), FAKE, 100, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_score_distance(ctypes.byref(d), FAKE, 0, FAKE, FAKE, None) == tri.TRI_ERR_INVALID
+    o = _opts()
+    step = lambda **kw: lib.tri_compress_step_distance(  # noqa: E731
+        ctypes.byref(d), kw.get("table", FAKE), kw.get("max_dist", 100), kw.get("pos", FAKE), ctypes.byref(kw.get("o", o)),
+        None, kw.get("freed", FAKE), kw.get("count", FAKE), None, FAKE, kw.get("ws", 1 << 40), None, None)
+    assert step(pos=None) == tri.TRI_ERR_INVALID
+    assert step(o=_opts(sinks=60)) == tri.TRI_ERR_INVALID
+    assert step(freed=None, count=None) == tri.TRI_ERR_INVALID
+    assert step(ws=64) == tri.TRI_ERR_WORKSPACE
