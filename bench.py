@@ -60,6 +60,8 @@ def parse_args():
     ap.add_argument("--trigger", type=int, default=0, help="compress only sequences longer than this (variant)")
     ap.add_argument("--aggregate", choices=["mean", "max"], default="mean",
                     help="GQA aggregation of the per-head scores (variant)")
+    ap.add_argument("--score-mode", choices=["keys", "distance"], default="keys",
+                    help="keys: score every cached key (the method); distance: table of the centres (variant)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling cases of the same kernels)")
     return ap.parse_args()
@@ -267,6 +269,7 @@ def run_ours(args, world, rank, local, dist):
     cache = tri.KvCache(wl.k_pool, wl.v_pool, wl.block_table, wl.seq_len, wl.cur_pos,
                         torch.zeros(1, dtype=torch.int32, device=dev), G)
     variant = (args.sinks, args.trigger, args.aggregate) != (0, 0, "mean")
+    distance = args.score_mode == "distance"
     opt = tri.step_options(B, W, args.sinks, args.trigger,
                            tri.TRI_AGG_MAX if args.aggregate == "max" else tri.TRI_AGG_MEAN)
     ws = tri.alloc_workspace(cache, opt)
@@ -279,15 +282,35 @@ def run_ours(args, world, rank, local, dist):
     save_v = wl.v_pool[:, rblocks].clone()
     save_len = wl.seq_len.clone()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    table_ms = None
+    if distance:
+        # one-time table of the centres (untimed, like the calibration)
+        max_dist = int(wl.cur_pos.max().item()) + 1
+        dtable = torch.empty(L, Hkv, max_dist + 1, device=dev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        tri.tri_distance_table(qbar, wl.key_centres.float().contiguous(), cfg.base, wl.deltas,
+                               tri.TRI_AGG_MAX if args.aggregate == "max" else tri.TRI_AGG_MEAN, dtable)
+        t1.record()
+        torch.cuda.synchronize(dev)
+        table_ms = t0.elapsed_time(t1)
+        max_len = wl.max_blocks * 16
+        slot_pos = torch.arange(max_len, dtype=torch.int32, device=dev).repeat(S, L, Hkv, 1).contiguous()
+        save_pos = slot_pos[..., :B].clone()
 
     def restore():
         wl.k_pool[:, rblocks] = save_k
         wl.v_pool[:, rblocks] = save_v
         wl.seq_len.copy_(save_len)
+        if distance:
+            slot_pos[..., :B] = save_pos
         flush.zero_()
 
     def step(events=None, idx_out=None):
-        if variant:
+        if distance:
+            tri.tri_compress_step_distance(cache, dtable, slot_pos, opt, ws, freed_ids=freed, freed_count=count,
+                                           idx_out=idx_out, events=events)
+        elif variant:
             tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, freed_ids=freed,
                                      freed_count=count, idx_out=idx_out, events=events)
         else:
@@ -352,14 +375,16 @@ def run_ours(args, world, rank, local, dist):
     ms_per_step = total_ms / args.steps
 
     peak, peak_kind = measured_peak()
-    k_bytes = keys_per_step * 256
+    bytes_per_key = 12 if distance else 256     # distance: position + table entry + score; keys: the bf16 key
+    k_bytes = keys_per_step * bytes_per_key
     moved_bytes = moved * 4 * 256
     score_mean = statistics.mean(score_ms)
     achieved = k_bytes / (score_mean / 1e3) / 1e9
     tpk = recorded_traffic_per_key()
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4), "traffic": (round(tpk * keys_per_step) if tpk else None),
-                "kernel": "score_kernel", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                "frac": round(achieved / peak, 4),
+                "traffic": (round(tpk * keys_per_step) if tpk and not variant and not distance else None),
+                "kernel": "distance_score_kernel" if distance else "score_kernel", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s",
                 "algorithmic_bytes_per_launch": k_bytes, "ms_per_launch": round(score_mean, 5),
                 "timing": f"CUDA events around the score kernel, {n_phase} live steps",
@@ -391,6 +416,7 @@ def run_ours(args, world, rank, local, dist):
         "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "seq_lens": lens,
                    "budget": B, "window": W, "rope_base": cfg.base, "deltas": wl.deltas,
                    "sinks": args.sinks, "trigger": trig, "aggregate": args.aggregate,
+                   "score_mode": args.score_mode, "distance_table_build_ms": table_ms,
                    "keys_per_step_per_gpu": keys_per_step, "freed_blocks_per_step": job_freed,
                    "parallelism": f"units sharded: one independent cache per GPU x{world}",
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
