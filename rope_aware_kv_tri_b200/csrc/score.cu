@@ -459,6 +459,8 @@ int score_heads_per_tile(int Hkv) {
 }
 
 cudaError_t launch_score(const ScoreParams& p_in, int max_items, int num_sms, cudaStream_t stream, bool pdl) {
+    if (p_in.agg_heads > 1 && !p_in.cuda_cores_only && score_mma_supported(p_in))
+        return launch_score_mma(p_in, max_items, num_sms, stream, pdl);
     ScoreParams p = p_in;
     int stages = kStageBudgetBytes / (p.heads_per_tile * kTileBytes);
     if (stages > kMaxStages) stages = kMaxStages;

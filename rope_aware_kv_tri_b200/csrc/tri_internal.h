@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "tri_attention.h"
@@ -85,10 +86,21 @@ struct ScoreParams {
     int L, Hkv, num_blocks, S, max_blocks;
     int heads_per_tile;       // HG, divides 8 and Hkv
     int agg_heads;            // 0: folded group mean; G: max over G per-head scores
+    int cuda_cores_only;      // 1: never the tensor-core max kernel
     int stages;
 };
 int score_heads_per_tile(int Hkv);
 cudaError_t launch_score(const ScoreParams& p, int max_items, int num_sms, cudaStream_t stream, bool pdl = false);
+
+// Max over the group with the dot products on the tensor cores (score_mma.cu):
+// G in {2, 4, 8}, Hkv a multiple of 8.  The K pool is read through a TMA
+// tensor map (2-D: 128 dims x all rows, 128-byte swizzle).
+struct MmaScoreParams {
+    ScoreParams base;
+    CUtensorMap tmap;
+};
+bool score_mma_supported(const ScoreParams& p);
+cudaError_t launch_score_mma(const ScoreParams& p, int max_items, int num_sms, cudaStream_t stream, bool pdl);
 
 // --------------------------------------------------- select + compaction
 struct EvictParams {

@@ -95,9 +95,23 @@ def test_select_trigger_keeps_short_units():
 
 # ----------------------------------------------------------------- score
 
-@pytest.mark.parametrize("name", ["cfg1", "hkv4", "cfg2s", "cfg5s"])      # G = 1, 2, 4, 8
+MAX_CASES = {
+    # CUDA-core kernel (G = 1, or KV heads not a multiple of 8)
+    "cfg1": SMALL["cfg1"],
+    "hkv4": SMALL["hkv4"],
+    "hkv4_g4": CONFIGS["cfg2"].replace(L=1, Hkv=4, G=4, lens=[1025, 300], n_samples=256, table="shuffled"),
+    "hkv2_g8": CONFIGS["cfg5"].replace(L=1, Hkv=2, G=8, lens=[777, 16, 0], n_samples=256),
+    # tensor-core kernel (8 KV heads per tile, G = 2, 4, 8)
+    "hkv8_g2": CONFIGS["cfg2"].replace(L=2, Hkv=8, G=2, lens=[2000, 700, 1], n_samples=256, table="shuffled"),
+    "cfg2s": SMALL["cfg2s"],
+    "cfg5s": SMALL["cfg5s"],
+    "hkv16_g4": CONFIGS["cfg2"].replace(L=1, Hkv=16, G=4, lens=[900, 33], n_samples=256, table="shuffled"),
+}
+
+
+@pytest.mark.parametrize("name", list(MAX_CASES))
 def test_score_max_over_group_matches_oracle(name):
-    wl = make_workload(SMALL[name], device=DEV, seed=4)
+    wl = make_workload(MAX_CASES[name], device=DEV, seed=4)
     stats = gpu_stats(wl)
     ref_stats = oracle_stats(wl)
     cache = cache_of(wl)
