@@ -442,10 +442,11 @@ tri_status tri_distance_table(int L, int Hkv, int G, int D, const float *qbar, c
 /*
  * tri_score_distance - scores[s][l][h][t] = table[l][h][cur_pos[s] - pos] with
  * pos = slot_pos[s][l][h][t], for t < seq_len[s]; the rest is not written.
- *   slot_pos : int32 [S][L][Hkv][max_blocks*16], the position each slot's key
- *              was cached at (slot_pos[...][t] = t for a cache never compacted)
+ *   slot_pos : int32 [S][L][Hkv][max_blocks*16], 16-byte aligned: the position
+ *              each slot's key was cached at (slot_pos[...][t] = t for a cache
+ *              never compacted)
  *   table, max_dist : as built by tri_distance_table for this cache's L, Hkv
- *   scores   : f32 [S][L][Hkv][max_blocks*16]
+ *   scores   : f32 [S][L][Hkv][max_blocks*16], 16-byte aligned
  * A distance outside [0, max_dist] raises TRI_DEVFLAG_BOUNDS (the nearest
  * table entry is used).  Errors: TRI_ERR_INVALID, TRI_ERR_UNSUPPORTED,
  * TRI_ERR_CUDA.

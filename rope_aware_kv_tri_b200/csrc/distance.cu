@@ -108,18 +108,34 @@ __global__ void __launch_bounds__(kDistThreads) distance_score_kernel(const Dist
     float* out = p.scores + (int64_t)u * p.score_stride;
     uint32_t lo = 0xffffffffu, hi = 0u;
     bool bad = false;
-    for (int t = t0 + threadIdx.x; t < t1; t += kDistThreads) {
-        int64_t d = P - (int64_t)pos[t];
+    auto score_one = [&](int32_t position) -> float {
+        int64_t d = P - (int64_t)position;
         if (d < 0 || d > p.max_dist) {
             bad = true;
             d = d < 0 ? 0 : p.max_dist;
         }
         const float v = __ldg(tab + d);
-        out[t] = v;
         const uint32_t key = order_key(v);
         lo = min(lo, key);
         hi = max(hi, key);
+        return v;
+    };
+    // Four slots per thread and step: one 16-byte position load, four
+    // independent table reads, one 16-byte score store (t0 and the unit rows
+    // are multiples of 4 slots, so both accesses are aligned).
+    const int n4 = (t1 - t0) >> 2;
+    const int4* pos4 = reinterpret_cast<const int4*>(pos + t0);
+    float4* out4 = reinterpret_cast<float4*>(out + t0);
+    for (int i = threadIdx.x; i < n4; i += kDistThreads) {
+        const int4 q = pos4[i];
+        float4 v;
+        v.x = score_one(q.x);
+        v.y = score_one(q.y);
+        v.z = score_one(q.z);
+        v.w = score_one(q.w);
+        out4[i] = v;
     }
+    for (int t = t0 + 4 * n4 + threadIdx.x; t < t1; t += kDistThreads) out[t] = score_one(pos[t]);
     if (__syncthreads_or(bad) && threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
     if (!p.unit_kmin) return;
     lo = __reduce_min_sync(0xffffffffu, lo);

@@ -316,7 +316,7 @@ DistScoreParams make_distance_params(const tri_kv_desc* desc, const float* table
 }
 
 tri_status check_distance_args(const float* table, int max_dist, const int32_t* slot_pos) {
-    if (!table || !slot_pos || !aligned(table, 4) || !aligned(slot_pos, 4)) return TRI_ERR_INVALID;
+    if (!table || !slot_pos || !aligned(table, 4) || !aligned(slot_pos, 16)) return TRI_ERR_INVALID;
     if (max_dist < 1 || max_dist >= (1 << 24)) return TRI_ERR_INVALID;
     return TRI_OK;
 }
@@ -567,7 +567,7 @@ tri_status tri_score_distance(const tri_kv_desc* desc, const float* table, int m
     tri_status st = check_desc(desc);
     if (st != TRI_OK) return st;
     if ((st = check_distance_args(table, max_dist, slot_pos)) != TRI_OK) return st;
-    if (!scores || !aligned(scores, 4)) return TRI_ERR_INVALID;
+    if (!scores || !aligned(scores, 16)) return TRI_ERR_INVALID;
     if (desc->S == 0) return TRI_OK;
     return cuda_status(launch_distance_score(make_distance_params(desc, table, max_dist, slot_pos, scores), stream));
 }

@@ -249,3 +249,9 @@ def test_distance_entries_reject(lib):
     assert step(o=_opts(sinks=60)) == tri.TRI_ERR_INVALID
     assert step(freed=None, count=None) == tri.TRI_ERR_INVALID
     assert step(ws=64) == tri.TRI_ERR_WORKSPACE
+
+
+def test_distance_alignment_rules(lib):
+    d = _desc()
+    assert lib.tri_score_distance(ctypes.byref(d), FAKE, 100, FAKE + 4, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_score_distance(ctypes.byref(d), FAKE, 100, FAKE, FAKE + 8, None) == tri.TRI_ERR_INVALID
