@@ -1,0 +1,76 @@
+"""ctypes wrapper of the plain C oracle (tri_oracle_c.c).
+
+TEST INFRASTRUCTURE: used by the tests and by the CPU legs of ``bench.py``
+(the CPU baseline and the reference arm) to time the oracle on every host
+core.  Built in-tree with gcc into ``oracle/_lib/libtrioracle.so``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import shutil
+import subprocess
+from typing import Sequence, Tuple
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "tri_oracle_c.c")
+LIB = os.path.join(HERE, "_lib", "libtrioracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle (plain -O2, no fast-math) if missing or stale."""
+    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+        return LIB
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        raise RuntimeError("no C compiler for the C oracle")
+    os.makedirs(os.path.dirname(LIB), exist_ok=True)
+    tmp = LIB + ".tmp"
+    subprocess.run([cc, "-O2", "-fPIC", "-shared", "-o", tmp, SRC, "-lm"], check=True, capture_output=True)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P, I = ctypes.c_void_p, ctypes.c_int
+        lib.tri_oracle_unit.restype = I
+        lib.tri_oracle_unit.argtypes = [P, P, I, I, P, P, P, I, ctypes.c_int64, P, I, ctypes.c_double, I, I,
+                                        P, P, P, P]
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> ctypes.c_void_p:
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def compress_unit_c(k_bits: np.ndarray, v_bits: np.ndarray, qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray,
+                    p: int, deltas: Sequence[int], base: float, budget: int,
+                    window: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray, np.ndarray]:
+    """One unit: k_bits / v_bits are bf16 bit patterns [T, D] (int16 or uint16),
+    statistics of its G query heads.  Returns (scores, idx, new K rows, new V rows)."""
+    lib = _load()
+    k = np.ascontiguousarray(k_bits).view(np.uint16)
+    v = np.ascontiguousarray(v_bits).view(np.uint16)
+    T, D = k.shape
+    qb = np.ascontiguousarray(qbar, dtype=np.float64)
+    qa = np.ascontiguousarray(qabs, dtype=np.float64)
+    r = np.ascontiguousarray(R, dtype=np.float64)
+    d = np.ascontiguousarray(np.asarray(deltas, dtype=np.int32))
+    scores = np.empty(T, dtype=np.float64)
+    idx = np.empty(max(min(T, budget), 1), dtype=np.int32)
+    ko, vo = np.empty_like(k), np.empty_like(v)
+    kept = lib.tri_oracle_unit(_ptr(k), _ptr(v), T, D, _ptr(qb), _ptr(qa), _ptr(r), qb.shape[0], int(p), _ptr(d),
+                               d.shape[0], float(base), int(budget), int(window), _ptr(scores), _ptr(idx), _ptr(ko),
+                               _ptr(vo))
+    if kept < 0:
+        raise ValueError("C oracle rejected its arguments")
+    return scores, idx[:kept].astype(np.int64), ko.view(k_bits.dtype), vo.view(v_bits.dtype)
