@@ -62,6 +62,8 @@ typedef int tri_status;
 #define TRI_ERR_TIMEOUT        5  /* a bounded device wait gave up            */
 #define TRI_ERR_NONFINITE      6  /* a NaN score was seen                     */
 #define TRI_ERR_WORKSPACE      7  /* workspace missing, small or misaligned   */
+/* TRI_ERR_FREELIST (8): a device free list was too short or full (see the
+ * free-list calls below). */
 
 /* Bits of the device status word. */
 #define TRI_DEVFLAG_BOUNDS     1
