@@ -62,6 +62,9 @@ def parse_args():
                     help="GQA aggregation of the per-head scores (variant)")
     ap.add_argument("--score-mode", choices=["keys", "distance"], default="keys",
                     help="keys: score every cached key (the method); distance: table of the centres (variant)")
+    ap.add_argument("--shard", choices=["sequences", "heads"], default="sequences",
+                    help="N>1: an independent cache per GPU (weak scaling) or the KV heads of one "
+                         "cache split over the GPUs (strong scaling)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling cases of the same kernels)")
     return ap.parse_args()
@@ -276,7 +279,11 @@ def run_ours(args, world, rank, local, dist):
         cfg = cfg.replace(L=args.layers, name=f"{cfg.name} (L={args.layers})")
     if args.workload == "cfg3":
         raise SystemExit("the decode-loop workload is measured by tests/test_gpu_workloads.py, not here")
-    from rope_aware_kv_tri_b200.sharding import reduce_job, shard_seed, keys_per_second
+    from rope_aware_kv_tri_b200.sharding import freed_consistent, keys_per_second, reduce_job, shard_heads, shard_seed
+    heads_mode = args.shard == "heads" and world > 1
+    if heads_mode:
+        # this rank's slice of the KV heads (and their query heads) of every sequence
+        cfg = cfg.replace(Hkv=len(shard_heads(cfg.Hkv, world, rank)))
     wl = make_workload(cfg, device=dev, seed=shard_seed(cfg.seed, rank) if world > 1 else cfg.seed)
     L, Hkv, G, Hq, S = cfg.L, cfg.Hkv, cfg.G, cfg.Hq, cfg.S
     B, W = cfg.budget, cfg.window
@@ -401,6 +408,7 @@ def run_ours(args, world, rank, local, dist):
     score_ms = [e[1].elapsed_time(e[2]) for e in pevs]
     evict_ms = [e[2].elapsed_time(e[3]) for e in pevs]
     total_ms, job_keys, job_freed = reduce_job(dist, sum(step_ms), keys_per_step, freed_per_step, dev)
+    freed_same = freed_consistent(dist, freed_per_step, dev) if heads_mode else None
     value = keys_per_second(job_keys, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
@@ -442,13 +450,15 @@ def run_ours(args, world, rank, local, dist):
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": "strong" if heads_mode else "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "seq_lens": lens,
                    "budget": B, "window": W, "rope_base": cfg.base, "deltas": wl.deltas,
                    "sinks": args.sinks, "trigger": trig, "aggregate": args.aggregate,
                    "score_mode": args.score_mode, "distance_table_build_ms": table_ms,
                    "keys_per_step_per_gpu": keys_per_step, "freed_blocks_per_step": job_freed,
-                   "parallelism": f"units sharded: one independent cache per GPU x{world}",
+                   "parallelism": (f"KV heads split over {world} GPUs ({cfg.Hkv} per GPU), freed-block "
+                                   f"counts all-reduced (equal on every rank: {freed_same})" if heads_mode else
+                                   f"units sharded: one independent cache per GPU x{world}"),
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
                    "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
                    "timing": "CUDA events around each tri_compress_step; kept-region restore and L2 flush "

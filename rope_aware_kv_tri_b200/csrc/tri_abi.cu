@@ -235,6 +235,35 @@ void record(cudaEvent_t ev, cudaStream_t stream) {
     if (ev) cudaEventRecord(ev, stream);
 }
 
+// The plan CTA's part of a step's query launch: lengths, work-item and
+// freed-list offsets, key ranges, scratch counters, the free-list reservation.
+void set_step_plan(QueryParams& q, const tri_kv_desc* desc, uint8_t* ws, const WsLayout& w, int budget, int trigger,
+                   int32_t* freed_count, const tri_free_list* free_list) {
+    q.L = desc->L;
+    q.Hkv = desc->Hkv;
+    q.G = desc->G;
+    q.S = desc->S;
+    q.seq_len = desc->seq_len;
+    q.max_blocks = desc->max_blocks;
+    q.heads_per_tile = score_heads_per_tile(desc->Hkv);
+    q.status = desc->status;
+    q.do_plan = 1;
+    q.budget = budget;
+    q.trigger = trigger;
+    q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
+    q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
+    q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
+    q.freed_count = freed_count;
+    q.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
+    q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
+    q.zero_words = reinterpret_cast<int32_t*>(ws + w.words);
+    if (free_list) {
+        q.fl_count = free_list->count;
+        q.fl_capacity = free_list->capacity;
+        q.fl_base = reinterpret_cast<int32_t*>(ws + w.words) + 2;
+    }
+}
+
 // The selection and compaction launches of a step, after its scores are in
 // the workspace (evict: select + plan + at-risk rows; copy-out; move).
 tri_status select_and_compact(const tri_kv_desc* desc, uint8_t* ws, const WsLayout& w, const tri_step_options& opt,
@@ -500,21 +529,7 @@ tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const floa
     QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
                                       reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
     q.per_head = per_head ? 1 : 0;
-    q.do_plan = 1;
-    q.budget = budget;
-    q.trigger = trigger;
-    q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
-    q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
-    q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
-    q.freed_count = freed_count;
-    q.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
-    q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
-    q.zero_words = reinterpret_cast<int32_t*>(ws + w.words);
-    if (free_list) {
-        q.fl_count = free_list->count;
-        q.fl_capacity = free_list->capacity;
-        q.fl_base = reinterpret_cast<int32_t*>(ws + w.words) + 2;
-    }
+    set_step_plan(q, desc, ws, w, budget, trigger, freed_count, free_list);
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     if (events) record(events->after_query, stream);
 
@@ -597,30 +612,8 @@ tri_status tri_compress_step_distance(tri_kv_desc* desc, const float* table, int
     const WsLayout w = ws_layout(desc, budget);
     const int trigger = effective_trigger(*opt);
     QueryParams q{};
-    q.L = desc->L;
-    q.Hkv = desc->Hkv;
-    q.G = desc->G;
-    q.S = desc->S;
-    q.seq_len = desc->seq_len;
-    q.max_blocks = desc->max_blocks;
-    q.heads_per_tile = score_heads_per_tile(desc->Hkv);
-    q.status = desc->status;
-    q.plan_only = 1;
-    q.do_plan = 1;
-    q.budget = budget;
-    q.trigger = trigger;
-    q.len_ws = reinterpret_cast<int32_t*>(ws + w.len_ws);
-    q.item_off = reinterpret_cast<int32_t*>(ws + w.item_off);
-    q.freed_off = reinterpret_cast<int32_t*>(ws + w.freed_off);
-    q.freed_count = freed_count;
-    q.unit_kmin = reinterpret_cast<uint32_t*>(ws + w.kmin);
-    q.unit_kmax = reinterpret_cast<uint32_t*>(ws + w.kmax);
-    q.zero_words = reinterpret_cast<int32_t*>(ws + w.words);
-    if (free_list) {
-        q.fl_count = free_list->count;
-        q.fl_capacity = free_list->capacity;
-        q.fl_base = reinterpret_cast<int32_t*>(ws + w.words) + 2;
-    }
+    q.plan_only = 1;       // the distance table replaces the effective queries
+    set_step_plan(q, desc, ws, w, budget, trigger, freed_count, free_list);
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     if (events) record(events->after_query, stream);
     const bool pdl = events == nullptr;

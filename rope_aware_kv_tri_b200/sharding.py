@@ -22,6 +22,33 @@ def shard_sequences(num_sequences: int, world: int, rank: int) -> List[int]:
     return list(range(rank, num_sequences, world))
 
 
+def shard_heads(num_kv_heads: int, world: int, rank: int) -> List[int]:
+    """KV heads owned by ``rank`` when the heads are split across GPUs (as a
+    tensor-parallel KV cache is): a contiguous slice of Hkv / world heads.
+    Every sequence lives on every rank; each rank compresses its own heads
+    in its own paged pool, and since every head keeps the same budget the
+    ranks free the same number of blocks per sequence."""
+    if world < 1 or not (0 <= rank < world):
+        raise ValueError("need world >= 1 and 0 <= rank < world")
+    if num_kv_heads % world:
+        raise ValueError("the KV heads must divide evenly over the ranks")
+    per = num_kv_heads // world
+    return list(range(rank * per, (rank + 1) * per))
+
+
+def freed_consistent(dist, freed_this_rank: int, device=None) -> bool:
+    """Head sharding: all-reduce the freed-block count (min and max over the
+    ranks) and return whether every rank freed the same number."""
+    import torch
+    if dist is None:
+        return True
+    lo = torch.tensor([int(freed_this_rank)], dtype=torch.int64, device=device)
+    hi = lo.clone()
+    dist.all_reduce(lo, op=dist.ReduceOp.MIN)
+    dist.all_reduce(hi, op=dist.ReduceOp.MAX)
+    return int(lo.item()) == int(hi.item())
+
+
 def shard_seed(base_seed: int, rank: int) -> int:
     """Seed of a rank's synthetic cache (independent streams per rank)."""
     return int(base_seed) * 1000003 + int(rank)

@@ -14,8 +14,8 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-from rope_aware_kv_tri_b200.sharding import (check_partition, keys_per_second, reduce_job, shard_seed,
-                                             shard_sequences)
+from rope_aware_kv_tri_b200.sharding import (check_partition, freed_consistent, keys_per_second, reduce_job,
+                                             shard_heads, shard_seed, shard_sequences)
 
 
 def _free_port():
@@ -72,3 +72,45 @@ def test_single_process_reduction_and_errors():
     with pytest.raises(ValueError):
         keys_per_second(10, 1, 0.0)
     assert not check_partition([[0, 1], [1]], 2)
+
+
+def _heads_worker(rank, world, port, out, freed_by_rank):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        mine = shard_heads(8, world, rank)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, mine)
+        same = freed_consistent(dist, freed_by_rank[rank])
+        t, k, f = reduce_job(dist, 5.0 + rank, 100 * len(mine), freed_by_rank[rank])
+        out[rank] = (gathered, same, t, k, f)
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("freed_by_rank,consistent", [((30, 30), True), ((30, 29), False)])
+def test_two_ranks_head_sharding_and_freed_all_reduce(freed_by_rank, consistent):
+    world = 2
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    port = _free_port()
+    procs = [ctx.Process(target=_heads_worker, args=(r, world, port, out, freed_by_rank)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    heads = out[0][0]
+    assert heads == out[1][0] == [[0, 1, 2, 3], [4, 5, 6, 7]]
+    assert out[0][1] is consistent and out[1][1] is consistent
+    assert out[0][2] == out[1][2] == 6.0
+    assert out[0][3] == 800 and out[0][4] == sum(freed_by_rank)
+
+
+def test_head_sharding_rules():
+    assert shard_heads(8, 1, 0) == list(range(8))
+    assert shard_heads(8, 8, 3) == [3]
+    with pytest.raises(ValueError):
+        shard_heads(8, 3, 0)
+    assert freed_consistent(None, 5)
