@@ -265,6 +265,31 @@ __device__ __forceinline__ int lin_bucket(float x, float lo, float scale) {
     return b < 0 ? 0 : (b > kLinBins - 1 ? kLinBins - 1 : b);
 }
 
+// Emit the set bits of `bits` (nwords words, slot 32w + b) into sidx in
+// ascending order, at most `take` of them.  Each warp takes a contiguous run
+// of words; lane i tests bit i of the warp's current word, so the warp writes
+// a whole word per step whatever its population.
+__device__ void emit_kept(const uint32_t* bits, int nwords, int take, int* sidx, EvictSmem& sm) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per = (nwords + kEvictWarps - 1) / kEvictWarps;
+    const int w0 = min(warp * per, nwords), w1 = min(w0 + per, nwords);
+    int cnt = 0;
+    for (int w = w0 + lane; w < w1; w += 32) cnt += __popc(bits[w]);
+    cnt = __reduce_add_sync(0xffffffffu, cnt);
+    if (lane == 0) sm.warp_a[warp] = cnt;
+    __syncthreads();
+    int base = 0;
+    for (int k = 0; k < warp; ++k) base += sm.warp_a[k];
+    const uint32_t lt = lanemask_lt();
+    for (int w = w0; w < w1; ++w) {
+        const uint32_t kw = bits[w];
+        const int pos = base + __popc(kw & lt);
+        if (((kw >> lane) & 1u) && pos < take) sidx[pos] = w * 32 + lane;
+        base += __popc(kw);
+    }
+    __syncthreads();
+}
+
 // The cut from the list of the cut bucket's keys (rem = the cut's rank in
 // the bucket), then the kept candidates from the bitmaps: gt_bits holds the
 // candidates above the bucket; the list's keys above the cut join them, the
@@ -315,7 +340,6 @@ __device__ void finish_from_list(const uint32_t* list_key, const int* list_slot,
     for (int w = w0; w < w1; ++w) my_eq += __popc(eq_bits[w]);
     int tot;
     int eq_before = block_exclusive_scan<kEvictThreads>(my_eq, sm.scan_tmp, tot);
-    int my_keep = 0;
     for (int w = w0; w < w1; ++w) {
         uint32_t e = eq_bits[w];
         int allow = need_eq - eq_before;
@@ -327,21 +351,10 @@ __device__ void finish_from_list(const uint32_t* list_key, const int* list_slot,
             e ^= low;
             --allow;
         }
-        const uint32_t kw = gt_bits[w] | keep_e;
-        gt_bits[w] = kw;
-        my_keep += __popc(kw);
-    }
-    int off = block_exclusive_scan<kEvictThreads>(my_keep, sm.scan_tmp, tot);
-    for (int w = w0; w < w1; ++w) {
-        uint32_t kw = gt_bits[w];
-        while (kw) {
-            const int b = __ffs(kw) - 1;
-            if (off < take) sidx[off] = w * 32 + b;
-            ++off;
-            kw &= kw - 1u;
-        }
+        gt_bits[w] |= keep_e;
     }
     __syncthreads();
+    emit_kept(gt_bits, nwords, take, sidx, sm);
 }
 
 // One streaming pass (cand <= kCodeSlots): the histogram pass also keeps
