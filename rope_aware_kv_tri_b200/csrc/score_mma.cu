@@ -432,6 +432,16 @@ __device__ void mma_issue(const ScoreParams& p, const Smem& sm, uint32_t tmem_ba
         }
         tc_fence_after();
         if (m.ord != cur_ord) {
+            // The buffers of set m.ord were last used by set m.ord - 2, whose
+            // stages may be as recent as k - 2: wait until every stage before
+            // k has been read by its epilogue (so its products are done too).
+            for (uint32_t d = 1; cur_ord >= 0 && d < kGroups && d <= k; ++d) {
+                if (!warp_wait(&sm.tempty[(k - d) % kGroups], ((k - d) / kGroups) & 1u, abort_flag, lane)) {
+                    give_up(p, abort_flag);
+                    return;
+                }
+            }
+            tc_fence_after();
             write_coefficients<G>(p, m.unit0, sm.cbuf + (size_t)(m.ord & 1) * Sh::kCBytes,
                                   sm.wbuf + (size_t)(m.ord & 1) * (Sh::kWBytes / 4), lane);
             fence_proxy_async_smem();      // the products read C through the async proxy
