@@ -278,7 +278,7 @@ def run_ours(args, world, rank, local, dist):
     if args.layers > 0:
         cfg = cfg.replace(L=args.layers, name=f"{cfg.name} (L={args.layers})")
     if args.workload == "cfg3":
-        raise SystemExit("the decode-loop workload is measured by tests/test_gpu_workloads.py, not here")
+        return run_decode(args, world, rank, local, dist, cfg)
     from rope_aware_kv_tri_b200.sharding import freed_consistent, keys_per_second, reduce_job, shard_heads, shard_seed
     heads_mode = args.shard == "heads" and world > 1
     if heads_mode:
@@ -465,6 +465,84 @@ def run_ours(args, world, rank, local, dist):
                              "untimed; per-phase times from a separate live loop with phase events"},
         "roofline": roofline, "step_roofline": step_roofline,
         "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 5 * args.steps, "clocks": clk,
+    }
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_decode(args, world, rank, local, dist, cfg):
+    """The decode-loop workload: sequences of drawn lengths in one shared
+    paged pool; each round appends cfg.decode_append tokens to every
+    sequence (blocks popped from the device free list by tri_reserve_blocks,
+    rows written untimed), then one timed tri_compress_step_ex compresses
+    every sequence and pushes the freed blocks back on the device list.  The
+    host never reads freed ids.  Reports every round."""
+    import torch
+    import rope_aware_kv_tri_b200 as tri
+    from workload import make_workload
+    from workload.gen import write_tokens
+    from rope_aware_kv_tri_b200.sharding import keys_per_second, reduce_job, shard_seed
+    dev = torch.device("cuda", local)
+    wl = make_workload(cfg, device=dev, seed=shard_seed(cfg.seed, rank) if world > 1 else cfg.seed)
+    L, Hkv, G, Hq, S = cfg.L, cfg.Hkv, cfg.G, cfg.Hq, cfg.S
+    B, W = cfg.budget, cfg.window
+    qbar = torch.empty(L, Hq, 128, device=dev)
+    qabs = torch.empty(L, Hq, 64, device=dev)
+    R = torch.empty(L, Hq, device=dev)
+    tri.tri_calibrate_centers(wl.q_samples, qbar, qabs, R)
+    cache = tri.KvCache(wl.k_pool, wl.v_pool, wl.block_table, wl.seq_len, wl.cur_pos,
+                        torch.zeros(1, dtype=torch.int32, device=dev), G)
+    opt = tri.step_options(B, W, args.sinks, args.trigger)
+    ws = tri.alloc_workspace(cache, opt)
+    fl = tri.FreeList.from_ids(wl.free_blocks, wl.num_blocks, dev)
+    n_new = torch.full((S,), cfg.decode_append, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    rounds, total_ms, total_keys = [], 0.0, 0
+    clocks = ClockSampler(local)
+    clocks.start()
+    for r in range(cfg.decode_rounds):
+        tri.tri_reserve_blocks(cache, n_new, fl)
+        lens = wl.seq_len.tolist()
+        for s in range(S):
+            write_tokens(wl, s, lens[s], cfg.decode_append)
+        wl.seq_len += n_new
+        wl.cur_pos += cfg.decode_append
+        lens = wl.seq_len.tolist()
+        free_before = int(fl.count.item())
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record()
+        tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, free_list=fl)
+        b.record()
+        torch.cuda.synchronize(dev)
+        if tri.tri_sync_status(cache.status) != tri.TRI_OK:
+            raise RuntimeError(f"device status flag raised in decode round {r}")
+        ms = a.elapsed_time(b)
+        trig = max(args.trigger, B)
+        keys = sum(n for n in lens if n > trig) * L * Hkv
+        freed = int(fl.count.item()) - free_before
+        rounds.append({"round": r, "keys": keys, "ms": round(ms, 4), "keys_per_s": round(keys / (ms / 1e3), 1),
+                       "k_read_gbs": round(keys * 256 / (ms / 1e3) / 1e9, 1), "freed_blocks": freed,
+                       "mean_len_before": round(sum(lens) / S, 1)})
+        total_ms += ms
+        total_keys += keys
+    clocks.stop()
+    t_job, k_job, _ = reduce_job(dist, total_ms, total_keys, 0, dev)
+    value = keys_per_second(k_job, 1, t_job)
+    peak, peak_kind = measured_peak()
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": cfg.decode_rounds,
+        "warmup": 0, "ms_per_step": round(t_job / cfg.decode_rounds, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "sequences": S,
+                   "budget": B, "window": W, "append_per_round": cfg.decode_append,
+                   "free_list": "device (tri_reserve_blocks pops, the step pushes; no host read of freed ids)",
+                   "timing": "CUDA events around each round's tri_compress_step_ex; appends untimed",
+                   "rounds": rounds},
+        "roofline": {"bound": "hbm", "peak": peak, "unit": "GB/s", "peak_source": peak_kind,
+                     "achieved_k_read_first_round": rounds[0]["k_read_gbs"] if rounds else None},
+        "gpu_launches": 5 * cfg.decode_rounds, "clocks": clocks.summary(),
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
