@@ -65,6 +65,8 @@ def parse_args():
     ap.add_argument("--shard", choices=["sequences", "heads"], default="sequences",
                     help="N>1: an independent cache per GPU (weak scaling) or the KV heads of one "
                          "cache split over the GPUs (strong scaling)")
+    ap.add_argument("--phases", action="store_true",
+                    help="decode loop: time each round's phases with library events (serialises launches)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling cases of the same kernels)")
     return ap.parse_args()
@@ -511,9 +513,10 @@ def run_decode(args, world, rank, local, dist, cfg):
         free_before = int(fl.count.item())
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        pev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if args.phases else None
         torch.cuda.synchronize(dev)
         a.record()
-        tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, free_list=fl)
+        tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, free_list=fl, events=pev)
         b.record()
         torch.cuda.synchronize(dev)
         if tri.tri_sync_status(cache.status) != tri.TRI_OK:
@@ -525,6 +528,10 @@ def run_decode(args, world, rank, local, dist, cfg):
         rounds.append({"round": r, "keys": keys, "ms": round(ms, 4), "keys_per_s": round(keys / (ms / 1e3), 1),
                        "k_read_gbs": round(keys * 256 / (ms / 1e3) / 1e9, 1), "freed_blocks": freed,
                        "mean_len_before": round(sum(lens) / S, 1)})
+        if pev is not None:
+            rounds[-1]["phase_ms"] = {"query": round(pev[0].elapsed_time(pev[1]), 4),
+                                      "score": round(pev[1].elapsed_time(pev[2]), 4),
+                                      "select_compact": round(pev[2].elapsed_time(pev[3]), 4)}
         total_ms += ms
         total_keys += keys
     clocks.stop()

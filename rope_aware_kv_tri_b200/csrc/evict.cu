@@ -117,6 +117,13 @@ static_assert(sizeof(SelectScratch) >= TRI_MAX_BUDGET * sizeof(int), "position s
 
 // rows per ordered compaction round, staged in the selection scratch
 constexpr int kStageRows = (int)(sizeof(SelectScratch) / (2 * kRowBytes));
+// With many units per launch (several waves of CTAs), units whose at-risk
+// prefix is longer than a few ordered rounds compact it in place: the
+// scratch path moves those rows twice (out to the scratch and back), the
+// ordered rounds once, and the other units' CTAs hide the rounds' latency.
+// With one wave of units the longest in-place unit would set the kernel's
+// time, so every prefix that fits takes the scratch.
+constexpr int kScratchMaxRows = 4 * kStageRows;
 
 __device__ __forceinline__ int block_sum(int v, EvictSmem& sm) {
     int total;
@@ -930,12 +937,14 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
         const int m0 = block_sum(fixed, sm);     // idx_j == j exactly for j < m0
         const int J = block_sum(low, sm);        // idx_j < kept exactly for j < J
         // Rows [m0, J) read sources that compaction overwrites.  With a
-        // scratch area they are copied out first (copy-out kernel) and all
-        // rows then move independently (move kernel); otherwise, or if the
-        // scratch is full, this CTA moves them in place in ordered rounds
-        // and the move kernel moves only rows [J, kept).
+        // scratch area and a short prefix they are copied out first
+        // (copy-out kernel) and all rows then move independently (move
+        // kernel); otherwise (a long prefix, or the scratch is full) this CTA
+        // moves them in place in ordered rounds and the move kernel moves
+        // only rows [J, kept).
         int mode = kModeInPlace, off = 0;
-        if (p.unit_info && J > m0) {
+        const bool reserved = p.unit_info && J > m0 && (!p.many_units || J - m0 <= kScratchMaxRows);
+        if (reserved) {
             if (threadIdx.x == 0) sm.bcast[0] = atomicAdd(p.scratch_used, J - m0);
             __syncthreads();
             off = sm.bcast[0];
@@ -949,7 +958,7 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
                 p.scratch_owner[off + r] = u;
                 p.scratch_owner[p.scratch_rows + off + r] = sidx[m0 + r];
             }
-        } else if (p.unit_info && J > m0) {
+        } else if (reserved) {
             // the reservation overflowed: its rows inside the scratch stay unowned
             for (int r = off + threadIdx.x; r < min(off + (J - m0), p.scratch_rows); r += kEvictThreads)
                 p.scratch_owner[r] = -1;

@@ -296,6 +296,8 @@ tri_status select_and_compact(const tri_kv_desc* desc, uint8_t* ws, const WsLayo
     e.unit_info = reinterpret_cast<int32_t*>(ws + w.info);
     e.scratch_owner = reinterpret_cast<int32_t*>(ws + w.owner);
     e.scratch_rows = w.scratch_rows;
+    // the evict kernel keeps two 512-thread CTAs per SM resident
+    e.many_units = (int64_t)desc->S * desc->L * desc->Hkv > (int64_t)4 * device_sm_count() ? 1 : 0;
     tri_status st;
     if ((st = cuda_status(launch_evict(e, stream, pdl))) != TRI_OK) return st;
     MoveParams mv = make_move_params(desc, reinterpret_cast<const int32_t*>(ws + w.idx), budget);

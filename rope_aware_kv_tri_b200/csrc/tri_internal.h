@@ -136,6 +136,7 @@ struct EvictParams {
     int32_t* unit_info;        // [U][4]: m0, J, mode, scratch row
     int32_t* scratch_owner;    // [2][scratch_rows]: unit and source row of each scratch row
     int scratch_rows;          // capacity of the scratch in rows
+    int many_units;            // several waves of unit CTAs: long at-risk prefixes compact in place
 };
 cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream, bool pdl = false);
 
