@@ -65,6 +65,8 @@ def parse_args():
     ap.add_argument("--shard", choices=["sequences", "heads"], default="sequences",
                     help="N>1: an independent cache per GPU (weak scaling) or the KV heads of one "
                          "cache split over the GPUs (strong scaling)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--phases", action="store_true",
                     help="decode loop: time each round's phases with library events (serialises launches)")
     ap.add_argument("--layers", type=int, default=0,
@@ -377,6 +379,21 @@ def run_ours(args, world, rank, local, dist):
     if dist is not None:
         dist.barrier()
 
+    # Optionally the step as a CUDA graph: one capture, replayed every timed
+    # step (the same device pointers, so the replay redoes the whole step).
+    graph = None
+    if args.graph:
+        restore()
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        torch.cuda.synchronize(dev)
+        for _ in range(args.warmup):
+            restore()
+            graph.replay()
+        torch.cuda.synchronize(dev)
+
     # Timed steps: one event pair around each tri_compress_step (its kernels
     # then overlap their launches programmatically).
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
@@ -388,12 +405,16 @@ def run_ours(args, world, rank, local, dist):
     for k in range(args.steps):
         restore()
         evs[k][0].record()
-        step()
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
         evs[k][1].record()
     torch.cuda.synchronize(dev)
     if dist is not None:
         dist.barrier()
     clocks.stop()
+    del graph
     if tri.tri_sync_status(cache.status) != tri.TRI_OK:
         raise RuntimeError("device status flag raised during the timed steps")
     step_ms = [e[0].elapsed_time(e[1]) for e in evs]
@@ -463,6 +484,7 @@ def run_ours(args, world, rank, local, dist):
                                    f"units sharded: one independent cache per GPU x{world}"),
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
                    "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
+                   "launch": "CUDA graph replay of one captured step" if args.graph else "direct calls",
                    "timing": "CUDA events around each tri_compress_step; kept-region restore and L2 flush "
                              "untimed; per-phase times from a separate live loop with phase events"},
         "roofline": roofline, "step_roofline": step_roofline,

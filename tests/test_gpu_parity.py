@@ -364,3 +364,46 @@ def test_compress_step_prefix_heavy_units_mix_scratch_and_in_place():
     ek, ev = expected_pools_after(pk, pv, wl.block_table, lens, idx, kept)
     assert torch.equal(wl.k_pool.view(torch.int16), ek.view(torch.int16))
     assert torch.equal(wl.v_pool.view(torch.int16), ev.view(torch.int16))
+
+
+def test_compress_step_replays_from_a_cuda_graph():
+    """One step captured in a CUDA graph (its launches with programmatic
+    dependencies become graph edges) and replayed on a restored cache gives
+    the same cache, lengths, freed blocks and kept slots as a direct call."""
+    wl = _workload("cfg5s", seed=21)
+    stats = gpu_stats(wl)
+    budget, window = wl.cfg.budget, wl.cfg.window
+    S, L, Hkv = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv
+    cache = cache_of(wl)
+    ws = tri.alloc_workspace(cache, budget)
+    freed = torch.zeros(S * wl.max_blocks, dtype=torch.int32, device=DEV)
+    count = torch.zeros(1, dtype=torch.int32, device=DEV)
+    idx = torch.full((S, L, Hkv, budget), -7, dtype=torch.int32, device=DEV)
+    k0, v0, len0 = wl.k_pool.clone(), wl.v_pool.clone(), wl.seq_len.clone()
+
+    def step():
+        tri.tri_compress_step(cache, *stats, wl.cfg.base, wl.deltas, budget, window, freed, count, ws, idx_out=idx)
+
+    step()
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    direct = (wl.k_pool.clone(), wl.v_pool.clone(), wl.seq_len.clone(), freed[:int(count.item())].clone(), idx.clone())
+    wl.k_pool.copy_(k0)
+    wl.v_pool.copy_(v0)
+    wl.seq_len.copy_(len0)
+    idx.fill_(-7)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    torch.cuda.synchronize()
+    # capture records the work without running it: the cache is still the original
+    assert torch.equal(wl.seq_len, len0)
+    g.replay()
+    torch.cuda.synchronize()
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    assert torch.equal(wl.k_pool.view(torch.int16), direct[0].view(torch.int16))
+    assert torch.equal(wl.v_pool.view(torch.int16), direct[1].view(torch.int16))
+    assert torch.equal(wl.seq_len, direct[2])
+    assert torch.equal(freed[:int(count.item())], direct[3])
+    assert torch.equal(idx, direct[4])
+    del g
