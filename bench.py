@@ -51,7 +51,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="cfg2", help="cfg1 | cfg2 | cfg4 | cfg5")
+    ap.add_argument("--workload", default="l32h8_t32k", help="head1_t4096 | l32h8_t32k | decode16 | l32h8_t128k | l64h8g8_4x64k")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -281,7 +281,7 @@ def run_ours(args, world, rank, local, dist):
     cfg = CONFIGS[args.workload]
     if args.layers > 0:
         cfg = cfg.replace(L=args.layers, name=f"{cfg.name} (L={args.layers})")
-    if args.workload == "cfg3":
+    if args.workload == "decode16":
         return run_decode(args, world, rank, local, dist, cfg)
     from rope_aware_kv_tri_b200.sharding import freed_consistent, keys_per_second, reduce_job, shard_heads, shard_seed
     heads_mode = args.shard == "heads" and world > 1

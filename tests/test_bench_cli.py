@@ -23,7 +23,7 @@ def _run(args, env_extra=None, timeout=300):
 
 
 def test_reference_arm_prints_the_contract_line():
-    r = _run(["--impl", "reference", "--workload", "cfg1", "--steps", "1", "--warmup", "1", "--cpu-seconds", "1"])
+    r = _run(["--impl", "reference", "--workload", "head1_t4096", "--steps", "1", "--warmup", "1", "--cpu-seconds", "1"])
     assert r.returncode == 0, r.stderr[-2000:]
     line = r.stdout.strip().splitlines()[-1]
     d = json.loads(line)
@@ -37,7 +37,7 @@ def test_reference_arm_prints_the_contract_line():
 
 
 def test_reference_arm_other_ranks_exit_quietly():
-    r = _run(["--impl", "reference", "--workload", "cfg1", "--steps", "1", "--warmup", "0"],
+    r = _run(["--impl", "reference", "--workload", "head1_t4096", "--steps", "1", "--warmup", "0"],
              env_extra={"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""

@@ -80,7 +80,7 @@ def _positions(wl, seed, gapped):
 
 
 def test_score_distance_is_a_lookup_and_flags_bad_distances():
-    wl = make_workload(SMALL["cfg5s"], device=DEV, seed=11)
+    wl = make_workload(SMALL["l2h8g8_ragged6"], device=DEV, seed=11)
     L, Hkv = wl.cfg.L, wl.cfg.Hkv
     pos = _positions(wl, 1, gapped={0, 2})
     max_dist = int(wl.cur_pos.max().item()) + 5
@@ -108,7 +108,7 @@ def test_score_distance_is_a_lookup_and_flags_bad_distances():
 
 @pytest.mark.parametrize("sinks,trigger", [(0, 0), (4, 0), (2, 600)])
 def test_compress_step_distance_matches_oracle(sinks, trigger):
-    wl = make_workload(SMALL["cfg5s"], device=DEV, seed=12)
+    wl = make_workload(SMALL["l2h8g8_ragged6"], device=DEV, seed=12)
     budget, window = wl.cfg.budget, wl.cfg.window
     S, L, Hkv, G = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv, wl.cfg.G
     pos = _positions(wl, 2, gapped={2, 5})

@@ -23,15 +23,15 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 SMALL = {
-    "cfg1": CONFIGS["cfg1"],
-    "cfg2s": CONFIGS["cfg2"].replace(L=2, lens=[3001], budget=512, window=64, n_samples=512),
-    "cfg5s": CONFIGS["cfg5"].replace(L=2, lens=[700, 33, 1001, 16, 0, 530], budget=512, window=64,
+    "head1_t4096": CONFIGS["head1_t4096"],
+    "l2h8g4_t3001": CONFIGS["l32h8_t32k"].replace(L=2, lens=[3001], budget=512, window=64, n_samples=512),
+    "l2h8g8_ragged6": CONFIGS["l64h8g8_4x64k"].replace(L=2, lens=[700, 33, 1001, 16, 0, 530], budget=512, window=64,
                                      n_samples=256, table="shuffled", pool_headroom=0.2),
-    "cfg4s": CONFIGS["cfg4"].replace(L=2, lens=[5000], budget=1024, window=256, n_samples=512),
-    "hkv6": CONFIGS["cfg2"].replace(L=2, Hkv=6, G=3, lens=[777, 1500], budget=300, window=20,
+    "l2h8g4_t5000": CONFIGS["l32h8_t128k"].replace(L=2, lens=[5000], budget=1024, window=256, n_samples=512),
+    "hkv6": CONFIGS["l32h8_t32k"].replace(L=2, Hkv=6, G=3, lens=[777, 1500], budget=300, window=20,
                                     n_samples=256, table="shuffled"),
-    "hkv4": CONFIGS["cfg2"].replace(L=1, Hkv=4, G=2, lens=[1025], budget=100, window=0, n_samples=256),
-    "hkv3": CONFIGS["cfg2"].replace(L=1, Hkv=3, G=5, lens=[401, 17], budget=64, window=64, n_samples=128,
+    "hkv4": CONFIGS["l32h8_t32k"].replace(L=1, Hkv=4, G=2, lens=[1025], budget=100, window=0, n_samples=256),
+    "hkv3": CONFIGS["l32h8_t32k"].replace(L=1, Hkv=3, G=5, lens=[401, 17], budget=64, window=64, n_samples=128,
                                     table="shuffled"),
 }
 
@@ -50,7 +50,7 @@ def _workload(name, seed=0):
 # --------------------------------------------------------------- calibrate
 
 def test_calibrate_matches_oracle():
-    cfg = CONFIGS["cfg2"].replace(L=2, lens=[16], n_samples=777)
+    cfg = CONFIGS["l32h8_t32k"].replace(L=2, lens=[16], n_samples=777)
     wl = make_workload(cfg, device=DEV)
     qbar, qabs, R = gpu_stats(wl)
     rb, ra, rr = oracle_stats(wl)
@@ -75,7 +75,7 @@ def test_calibrate_degenerate_samples():
 
 # ------------------------------------------------------------- build query
 
-@pytest.mark.parametrize("name", ["cfg1", "cfg5s", "hkv3"])
+@pytest.mark.parametrize("name", ["head1_t4096", "l2h8g8_ragged6", "hkv3"])
 def test_build_query_matches_oracle(name):
     wl = _workload(name)
     stats = gpu_stats(wl)
@@ -195,7 +195,7 @@ def test_select_nan_ranks_lowest_and_is_flagged():
 
 # ---------------------------------------------------------------- compact
 
-@pytest.mark.parametrize("name", ["cfg5s", "hkv6", "cfg1"])
+@pytest.mark.parametrize("name", ["l2h8g8_ragged6", "hkv6", "head1_t4096"])
 def test_compact_bit_exact_for_given_indices(name):
     wl = _workload(name, seed=5)
     budget, window = wl.cfg.budget, wl.cfg.window
@@ -275,7 +275,7 @@ def test_compress_step_matches_oracle(name):
 def test_compress_step_all_equal_scores_keeps_earliest():
     """Zero statistics make every score exactly 0: the step keeps the lowest
     slots plus the window, exactly as the oracle."""
-    wl = _workload("cfg5s", seed=2)
+    wl = _workload("l2h8g8_ragged6", seed=2)
     L, Hq = wl.cfg.L, wl.cfg.Hq
     zero = (torch.zeros(L, Hq, 128, device=DEV), torch.zeros(L, Hq, 64, device=DEV),
             torch.ones(L, Hq, device=DEV))
@@ -292,7 +292,7 @@ def test_compress_step_all_equal_scores_keeps_earliest():
 
 
 def test_compress_step_budget_one_and_second_call_is_noop():
-    wl = _workload("cfg2s", seed=3)
+    wl = _workload("l2h8g4_t3001", seed=3)
     stats = gpu_stats(wl)
     out = run_step(wl, stats, 1, 1)
     assert out["status"] == tri.TRI_OK and wl.seq_len.tolist() == [1]
@@ -302,19 +302,19 @@ def test_compress_step_budget_one_and_second_call_is_noop():
 
 
 def test_bad_block_id_is_flagged_not_followed():
-    wl = _workload("cfg5s", seed=4)
+    wl = _workload("l2h8g8_ragged6", seed=4)
     stats = gpu_stats(wl)
     wl.block_table[0, 3] = wl.num_blocks + 1000          # out of the pool
     wl.block_table[2, 0] = -5
     out = run_step(wl, stats, 512, 64)
     assert out["status"] == tri.TRI_ERR_DEVICE_BOUNDS
     # the context is intact: a clean call afterwards succeeds
-    wl2 = _workload("cfg2s", seed=4)
+    wl2 = _workload("l2h8g4_t3001", seed=4)
     assert run_step(wl2, gpu_stats(wl2), 512, 64)["status"] == tri.TRI_OK
 
 
 def test_sequence_longer_than_its_table_is_flagged():
-    wl = _workload("cfg2s", seed=6)
+    wl = _workload("l2h8g4_t3001", seed=6)
     stats = gpu_stats(wl)
     wl.seq_len[0] = wl.max_blocks * 16 + 1
     k0 = wl.k_pool.clone()
@@ -328,7 +328,7 @@ def test_compress_step_prefix_heavy_units_mix_scratch_and_in_place():
     the budget, so each unit's at-risk prefix is nearly B rows: the step's
     scratch (a quarter of the kept rows) fills up and later units compact
     their prefix in place.  Both paths must give the oracle's result."""
-    cfg = CONFIGS["cfg2"].replace(L=1, Hkv=4, G=2, lens=[700, 650], budget=256, window=16, n_samples=64,
+    cfg = CONFIGS["l32h8_t32k"].replace(L=1, Hkv=4, G=2, lens=[700, 650], budget=256, window=16, n_samples=64,
                                   table="shuffled")
     wl = make_workload(cfg, device=DEV, seed=7)
     L, Hkv, Hq = cfg.L, cfg.Hkv, cfg.Hq
@@ -370,7 +370,7 @@ def test_compress_step_replays_from_a_cuda_graph():
     """One step captured in a CUDA graph (its launches with programmatic
     dependencies become graph edges) and replayed on a restored cache gives
     the same cache, lengths, freed blocks and kept slots as a direct call."""
-    wl = _workload("cfg5s", seed=21)
+    wl = _workload("l2h8g8_ragged6", seed=21)
     stats = gpu_stats(wl)
     budget, window = wl.cfg.budget, wl.cfg.window
     S, L, Hkv = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv

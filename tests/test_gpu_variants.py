@@ -97,15 +97,15 @@ def test_select_trigger_keeps_short_units():
 
 MAX_CASES = {
     # CUDA-core kernel (G = 1, or KV heads not a multiple of 8)
-    "cfg1": SMALL["cfg1"],
+    "head1_t4096": SMALL["head1_t4096"],
     "hkv4": SMALL["hkv4"],
-    "hkv4_g4": CONFIGS["cfg2"].replace(L=1, Hkv=4, G=4, lens=[1025, 300], n_samples=256, table="shuffled"),
-    "hkv2_g8": CONFIGS["cfg5"].replace(L=1, Hkv=2, G=8, lens=[777, 16, 0], n_samples=256),
+    "hkv4_g4": CONFIGS["l32h8_t32k"].replace(L=1, Hkv=4, G=4, lens=[1025, 300], n_samples=256, table="shuffled"),
+    "hkv2_g8": CONFIGS["l64h8g8_4x64k"].replace(L=1, Hkv=2, G=8, lens=[777, 16, 0], n_samples=256),
     # tensor-core kernel (8 KV heads per tile, G = 2, 4, 8)
-    "hkv8_g2": CONFIGS["cfg2"].replace(L=2, Hkv=8, G=2, lens=[2000, 700, 1], n_samples=256, table="shuffled"),
-    "cfg2s": SMALL["cfg2s"],
-    "cfg5s": SMALL["cfg5s"],
-    "hkv16_g4": CONFIGS["cfg2"].replace(L=1, Hkv=16, G=4, lens=[900, 33], n_samples=256, table="shuffled"),
+    "hkv8_g2": CONFIGS["l32h8_t32k"].replace(L=2, Hkv=8, G=2, lens=[2000, 700, 1], n_samples=256, table="shuffled"),
+    "l2h8g4_t3001": SMALL["l2h8g4_t3001"],
+    "l2h8g8_ragged6": SMALL["l2h8g8_ragged6"],
+    "hkv16_g4": CONFIGS["l32h8_t32k"].replace(L=1, Hkv=16, G=4, lens=[900, 33], n_samples=256, table="shuffled"),
 }
 
 
@@ -149,7 +149,7 @@ VARIANTS = [
 
 @pytest.mark.parametrize("var", VARIANTS, ids=[f"s{v['sinks']}_t{v['trigger']}_a{v['aggregate']}" for v in VARIANTS])
 def test_compress_step_ex_matches_oracle(var):
-    wl = make_workload(SMALL["cfg5s"], device=DEV, seed=6)
+    wl = make_workload(SMALL["l2h8g8_ragged6"], device=DEV, seed=6)
     budget, window = wl.cfg.budget, wl.cfg.window
     opt = tri.step_options(budget, window, **var)
     agg = "max" if var["aggregate"] == tri.TRI_AGG_MAX else "mean"
@@ -241,7 +241,7 @@ def _expected_reserve(table, lens, n_new, free):
 
 
 def test_free_list_push_and_reserve():
-    wl = make_workload(SMALL["cfg5s"], device=DEV, seed=8)
+    wl = make_workload(SMALL["l2h8g8_ragged6"], device=DEV, seed=8)
     budget, window = wl.cfg.budget, wl.cfg.window
     NB = wl.k_pool.shape[1]
     free0 = _unused_blocks(wl)
@@ -284,7 +284,7 @@ def test_free_list_push_and_reserve():
 
 
 def test_free_list_push_without_room_is_flagged():
-    wl = make_workload(SMALL["cfg5s"], device=DEV, seed=9)
+    wl = make_workload(SMALL["l2h8g8_ragged6"], device=DEV, seed=9)
     budget, window = wl.cfg.budget, wl.cfg.window
     lens = wl.seq_len.cpu().tolist()
     kept = [min(n, budget) for n in lens]
@@ -310,7 +310,7 @@ def test_decode_loop_with_device_free_list_matches_oracle_world():
     list; the host never reads freed ids.  The oracle world uses the host
     allocator.  The worlds' block ids differ, so the rows of each unit are
     compared through each world's own table."""
-    cfg = CONFIGS["cfg3"].replace(L=2, Hkv=4, G=2, lens=[0] * 4, lens_range=(300, 700), budget=256, window=32,
+    cfg = CONFIGS["decode16"].replace(L=2, Hkv=4, G=2, lens=[0] * 4, lens_range=(300, 700), budget=256, window=32,
                                   decode_append=64, decode_rounds=5, n_samples=256)
     sinks, trigger = 4, 256 + 64
     cpu = make_workload(cfg, device="cpu")

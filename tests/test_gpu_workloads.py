@@ -35,7 +35,7 @@ def _built():
 
 
 def test_decode_loop_two_worlds():
-    cfg = CONFIGS["cfg3"].replace(L=2, Hkv=4, G=2, lens=[0] * 4, lens_range=(300, 700), budget=256, window=32,
+    cfg = CONFIGS["decode16"].replace(L=2, Hkv=4, G=2, lens=[0] * 4, lens_range=(300, 700), budget=256, window=32,
                                   decode_append=64, decode_rounds=4, n_samples=256)
     cpu = make_workload(cfg, device="cpu")
     G, budget, window = cfg.G, cfg.budget, cfg.window
@@ -160,12 +160,12 @@ def _full_size(name, sample_units, check_all_rows):
 
 
 def test_full_size_32L_8H_T32768_B2048():
-    _full_size("cfg2", sample_units=8, check_all_rows=True)
+    _full_size("l32h8_t32k", sample_units=8, check_all_rows=True)
 
 
 def test_full_size_long_context_T131072_B4096():
-    _full_size("cfg4", sample_units=4, check_all_rows=True)
+    _full_size("l32h8_t128k", sample_units=4, check_all_rows=True)
 
 
 def test_full_size_wide_64L_G8_4x65536():
-    _full_size("cfg5", sample_units=4, check_all_rows=False)
+    _full_size("l64h8g8_4x64k", sample_units=4, check_all_rows=False)

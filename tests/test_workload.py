@@ -13,7 +13,7 @@ def _small(name, **kw):
 
 
 def test_generator_is_deterministic():
-    cfg = _small("cfg2", L=2, lens=[300], n_samples=64)
+    cfg = _small("l32h8_t32k", L=2, lens=[300], n_samples=64)
     a, b = make_workload(cfg), make_workload(cfg)
     assert torch.equal(a.k_pool, b.k_pool) and torch.equal(a.v_pool, b.v_pool)
     assert torch.equal(a.q_samples, b.q_samples)
@@ -22,7 +22,7 @@ def test_generator_is_deterministic():
 
 
 def test_shapes_and_tables():
-    cfg = _small("cfg5", L=2, lens=[70, 33, 1, 16], n_samples=8)
+    cfg = _small("l64h8g8_4x64k", L=2, lens=[70, 33, 1, 16], n_samples=8)
     wl = make_workload(cfg)
     L, NB, Hkv, bs, D = wl.k_pool.shape
     assert (L, Hkv, bs, D) == (2, 8, 16, 128) and wl.k_pool.dtype == torch.bfloat16
@@ -40,7 +40,7 @@ def test_shapes_and_tables():
 
 def test_cached_keys_are_rotated_centred_draws():
     """Each cached key, rotated back by its position, lies near its head's centre."""
-    cfg = _small("cfg1", lens=[64])
+    cfg = _small("head1_t4096", lens=[64])
     wl = make_workload(cfg)
     keys = wl.k_pool[0, 0:4, 0].reshape(64, 128).double()
     back = rope_rotate_half(keys, -torch.arange(64, dtype=torch.float64), cfg.base)
@@ -50,14 +50,14 @@ def test_cached_keys_are_rotated_centred_draws():
 
 
 def test_direct_statistics():
-    wl = make_workload(CONFIGS["cfg1"])
+    wl = make_workload(CONFIGS["head1_t4096"])
     mag = torch.sqrt(wl.qbar[..., :64].double() ** 2 + wl.qbar[..., 64:].double() ** 2)
     torch.testing.assert_close(wl.qabs.double(), 1.2 * mag, rtol=1e-6, atol=0)
     assert abs(wl.R.item() - 1 / 1.2) < 1e-7
 
 
 def test_decode_append_and_recycle():
-    cfg = _small("cfg3", L=1, lens=[0, 0], lens_range=(40, 60), budget=32, window=8,
+    cfg = _small("decode16", L=1, lens=[0, 0], lens_range=(40, 60), budget=32, window=8,
                  decode_append=20, n_samples=8)
     wl = make_workload(cfg)
     old = wl.seq_len.tolist()

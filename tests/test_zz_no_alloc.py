@@ -26,8 +26,8 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 CASES = [
-    CONFIGS["cfg1"],
-    CONFIGS["cfg5"].replace(L=2, lens=[700, 33, 1001, 16, 0, 530], budget=512, window=64, n_samples=256),
+    CONFIGS["head1_t4096"],
+    CONFIGS["l64h8g8_4x64k"].replace(L=2, lens=[700, 33, 1001, 16, 0, 530], budget=512, window=64, n_samples=256),
 ]
 
 

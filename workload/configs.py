@@ -76,24 +76,24 @@ class WorkloadConfig:
 
 # 1 layer, 1 KV head, T = 4096 at positions 0..4095, next query at 4096;
 # E|q_i| = 1.2 |c_q,i| given directly; offsets 1..1024; B = 512, W = 64.
-CFG1 = WorkloadConfig(
+HEAD1_T4096 = WorkloadConfig(
     name="single-head T=4096 B=512", L=1, Hkv=1, G=1, D=128, base=1e4,
     lens=[4096], deltas=geometric_offsets(1024), budget=512, window=64,
     stats="direct", qabs_ratio=1.2, table="identity")
 
 # 32 layers x 8 KV heads, G = 4, one sequence of 32768, base 5e5,
 # R ~ U(0.6, 0.98), offsets 1..4096, B = 2048, W = 128, compress once.
-CFG2 = WorkloadConfig(
+L32H8_T32K = WorkloadConfig(
     name="32Lx8H G=4 T=32768 B=2048", L=32, Hkv=8, G=4, D=128, base=5e5,
     lens=[32768], deltas=geometric_offsets(4096), budget=2048, window=128,
     stats="samples", r_range=(0.6, 0.98), table="identity")
 
-# Decode loop: the CFG2 model, 16 sequences with lengths U(8K, 32K) in one
+# Decode loop: the L32H8_T32K model, 16 sequences with lengths U(8K, 32K) in one
 # shared pool of 16-token blocks with 10 % headroom; every 128 appended
 # tokens compress to B = 2048 and recycle the freed blocks
 # ([GeoTrick] "Solving the Memory Fragmentation Problem": compaction every
 # ~128 decode steps).
-CFG3 = WorkloadConfig(
+DECODE16 = WorkloadConfig(
     name="decode 16 seqs U(8K,32K) every 128 tokens B=2048", L=32, Hkv=8, G=4,
     D=128, base=5e5, lens=[0] * 16, deltas=geometric_offsets(4096),
     budget=2048, window=128, stats="samples", r_range=(0.6, 0.98),
@@ -102,7 +102,7 @@ CFG3 = WorkloadConfig(
 
 # Long context: one sequence of 131072, base 1e6, B = 4096, W = 256; 10 % of
 # query heads at R ~ 0.3 so the norm term dominates there.
-CFG4 = WorkloadConfig(
+L32H8_T128K = WorkloadConfig(
     name="32Lx8H G=4 T=131072 B=4096", L=32, Hkv=8, G=4, D=128, base=1e6,
     lens=[131072], deltas=geometric_offsets(4096), budget=4096, window=256,
     stats="samples", r_range=(0.6, 0.98), low_r_fraction=0.10,
@@ -110,9 +110,15 @@ CFG4 = WorkloadConfig(
 
 # Wide model: 64 layers x 8 KV heads, G = 8, batch 4 x 65536 in a paged pool,
 # R ~ U(0.3, 0.98), offsets 1..8192, B = 4096, W = 128.
-CFG5 = WorkloadConfig(
+L64H8G8_4X64K = WorkloadConfig(
     name="64Lx8H G=8 4x65536 B=4096", L=64, Hkv=8, G=8, D=128, base=1e6,
     lens=[65536] * 4, deltas=geometric_offsets(8192), budget=4096, window=128,
     stats="samples", r_range=(0.3, 0.98), table="shuffled")
 
-CONFIGS = {"cfg1": CFG1, "cfg2": CFG2, "cfg3": CFG3, "cfg4": CFG4, "cfg5": CFG5}
+CONFIGS = {
+    "head1_t4096": HEAD1_T4096,
+    "l32h8_t32k": L32H8_T32K,
+    "decode16": DECODE16,
+    "l32h8_t128k": L32H8_T128K,
+    "l64h8g8_4x64k": L64H8G8_4X64K,
+}
