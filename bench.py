@@ -236,6 +236,18 @@ def oracle_sample(units, stats_fn, deltas, base, budget, window, seconds, sinks=
     return keys_done, t_used, n
 
 
+def host_cpu_model():
+    """The host CPU's model name, as the kernel reports it."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def c_oracle_sample(units, stats_fn, deltas, base, budget, window, seconds, threads):
     """Time the plain C float64 oracle on units, ``threads`` units at a time
     on the host cores, until about ``seconds`` of wall time have passed.
@@ -665,12 +677,15 @@ def run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens):
     threads = os.cpu_count() or 1
     keys, secs, n = c_oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
                                     args.cpu_seconds, threads)
+    c1, cs1, cn1 = c_oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
+                                   min(3.0, args.cpu_seconds), 1)
     k1, s1, n1 = oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
                                min(4.0, args.cpu_seconds), args.sinks, args.aggregate)
     return {"value": round(keys / secs, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": (f"{n} random units of this workload ({keys} keys), plain C float64 oracle, one unit per "
                        f"host thread on {threads} threads (wall time; inputs prepared untimed)"),
-            "seconds": round(secs, 2),
+            "seconds": round(secs, 2), "cpu_model": host_cpu_model(),
+            "c_oracle_1_thread": {"value": round(c1 / cs1, 1), "units": cn1, "seconds": round(cs1, 2)},
             "numpy_oracle_1_thread": {"value": round(k1 / s1, 1), "units": n1, "seconds": round(s1, 2)}}
 
 
@@ -742,7 +757,7 @@ def run_reference(args, world, rank):
            "config": {"workload": cfg.name, "L": cfg.L, "Hkv": cfg.Hkv, "G": cfg.G, "D": 128,
                       "seq_lens": cfg.lens, "budget": cfg.budget, "window": cfg.window},
            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
-                            "sample": sample},
+                            "sample": sample, "cpu_model": host_cpu_model()},
            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
