@@ -176,6 +176,60 @@ def test_select_bit_exact_on_same_scores(budget, window):
             assert np.all(idx[s, 0, h, kept[s]:] == -1)
 
 
+def _spaced_runs(cand):
+    """64 evenly spaced runs of 32 slots over candidates [0, cand)."""
+    stride = (cand - 32) // 63
+    return np.concatenate([c * stride + np.arange(32) for c in range(64)])
+
+
+@pytest.mark.parametrize("budget,window", [(2048, 128), (256, 0), (4096, 256)])
+def test_select_structured_score_patterns(budget, window):
+    """Score patterns with structure along the slots - ramps, periodic
+    scores, far outliers packed into evenly spaced runs, a low floor in them,
+    and thousands of exact ties at the cut value - at lengths from one to
+    several shared-memory bitmaps' worth of candidates.  Every result is the
+    oracle's."""
+    rng = np.random.default_rng(budget + window)
+    lens = [8192 + window, 20000, 65536, 131000]
+    kinds = ["normal", "ramp", "periodic", "spaced_high", "spaced_low", "crowded_cut"]
+    S, L, Hkv = len(lens), 1, len(kinds)
+    max_blocks = -(-max(lens) // 16)
+    k = torch.zeros(1, 1, Hkv, 16, 128, dtype=torch.bfloat16, device=DEV)
+    cache = tri.KvCache(k, k.clone(), torch.zeros(S, max_blocks, dtype=torch.int32, device=DEV),
+                        torch.tensor(lens, dtype=torch.int32, device=DEV), torch.zeros(S, dtype=torch.int64, device=DEV),
+                        status_tensor(DEV), 1)
+    sc = np.full((S, L, Hkv, max_blocks * 16), np.nan, dtype=np.float32)
+    for s, n in enumerate(lens):
+        cand = n - window
+        runs = _spaced_runs(cand)
+        for h, kind in enumerate(kinds):
+            x = rng.normal(size=n)
+            if kind == "ramp":
+                x = np.arange(n) * 1e-3 + 0.01 * x
+            elif kind == "periodic":
+                x = np.sin(np.arange(n) * 2 * np.pi / 512) + 0.05 * x
+            elif kind == "spaced_high":       # half of every run far above everything else
+                x[runs[::2]] = 50 + x[runs[::2]]
+            elif kind == "spaced_low":        # the runs sit far below everything else
+                x[runs] = -50 + x[runs]
+            elif kind == "crowded_cut":       # thousands of exact ties at the cut value
+                x = rng.normal(size=n) - 10
+                hi = rng.choice(cand, budget // 2, replace=False)
+                x[hi] = 10 + rng.random(budget // 2)
+                rest = np.setdiff1d(np.arange(cand), hi)
+                x[rng.choice(rest, min(3 * budget, rest.size), replace=False)] = 1.0
+            sc[s, 0, h, :n] = x.astype(np.float32)
+    idx = torch.full((S, L, Hkv, budget), -7, dtype=torch.int32, device=DEV)
+    kept = torch.full((S,), -7, dtype=torch.int32, device=DEV)
+    tri.tri_select_topk(cache, torch.from_numpy(sc).to(DEV), budget, window, idx, kept)
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    idx = idx.cpu().numpy()
+    for s, n in enumerate(lens):
+        for h, kind in enumerate(kinds):
+            ref = oracle.select(sc[s, 0, h, :n].astype(np.float64), n, budget, window)
+            assert np.array_equal(idx[s, 0, h], ref), (n, kind)
+
+
 def test_select_nan_ranks_lowest_and_is_flagged():
     n, budget, window = 300, 40, 5
     rng = np.random.default_rng(3)
