@@ -33,6 +33,10 @@ SMALL = {
     "hkv4": CONFIGS["l32h8_t32k"].replace(L=1, Hkv=4, G=2, lens=[1025], budget=100, window=0, n_samples=256),
     "hkv3": CONFIGS["l32h8_t32k"].replace(L=1, Hkv=3, G=5, lens=[401, 17], budget=64, window=64, n_samples=128,
                                     table="shuffled"),
+    # the largest budget the library takes (its kept-slot list fills 64 KiB of
+    # the selection CTA's shared memory); one sequence exactly at the budget
+    "l1h2g2_b16384": CONFIGS["l32h8_t32k"].replace(L=1, Hkv=2, G=2, lens=[40000, 16384, 20000], budget=16384,
+                                             window=1024, n_samples=256, table="shuffled"),
 }
 
 
@@ -182,7 +186,7 @@ def _spaced_runs(cand):
     return np.concatenate([c * stride + np.arange(32) for c in range(64)])
 
 
-@pytest.mark.parametrize("budget,window", [(2048, 128), (256, 0), (4096, 256)])
+@pytest.mark.parametrize("budget,window", [(2048, 128), (256, 0), (4096, 256), (16384, 1024)])
 def test_select_structured_score_patterns(budget, window):
     """Score patterns with structure along the slots - ramps, periodic
     scores, far outliers packed into evenly spaced runs, a low floor in them,
@@ -225,9 +229,11 @@ def test_select_structured_score_patterns(budget, window):
     assert tri.tri_sync_status(cache.status) == tri.TRI_OK
     idx = idx.cpu().numpy()
     for s, n in enumerate(lens):
+        k = min(n, budget)
         for h, kind in enumerate(kinds):
             ref = oracle.select(sc[s, 0, h, :n].astype(np.float64), n, budget, window)
-            assert np.array_equal(idx[s, 0, h], ref), (n, kind)
+            assert np.array_equal(idx[s, 0, h, :k], ref), (n, kind)
+            assert np.all(idx[s, 0, h, k:] == -1)
 
 
 def test_select_nan_ranks_lowest_and_is_flagged():
