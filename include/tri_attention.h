@@ -481,6 +481,21 @@ tri_status tri_sync_status(int32_t *status, cudaStream_t stream);
 /* Static, human-readable name of a status code. */
 const char *tri_status_string(tri_status s);
 
+/*
+ * tri_selftest_bounded_wait - test aid for the device error contract: one
+ * thread runs a device wait that nothing completes, under the same rule as
+ * every wait of the library's kernels (it gives up after 2 s), then ORs
+ * TRI_DEVFLAG_TIMEOUT into *status; tri_sync_status() then returns
+ * TRI_ERR_TIMEOUT and the context stays usable.
+ *   status : device int32 status word (caller-owned, 4-byte aligned).
+ *   flag   : null - wait on a shared-memory barrier that never completes;
+ *            else a device int32 the wait polls (acquire, GPU scope) and
+ *            that ends the wait as soon as it is non-zero (no timeout then).
+ * Returns TRI_ERR_INVALID for a null or misaligned status or flag,
+ * TRI_ERR_CUDA if the launch fails, else TRI_OK (asynchronous on `stream`).
+ */
+tri_status tri_selftest_bounded_wait(int32_t *status, const int32_t *flag, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

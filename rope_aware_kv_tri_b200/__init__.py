@@ -44,7 +44,7 @@ EXPORTS = (
     "tri_select_topk", "tri_compact_kv", "tri_compress_step", "tri_compress_step_static_scratch",
     "tri_sync_status", "tri_status_string", "tri_workspace_size_ex", "tri_score_ex", "tri_select_topk_ex",
     "tri_compress_step_ex", "tri_reserve_blocks", "tri_distance_table", "tri_score_distance",
-    "tri_compress_step_distance",
+    "tri_compress_step_distance", "tri_selftest_bounded_wait",
 )
 TRI_STATIC_SCRATCH_BYTES = 16 << 20
 
@@ -158,6 +158,7 @@ def _load() -> ctypes.CDLL:
                                            ctypes.POINTER(TriFreeList), P, P, P, P, S,
                                            ctypes.POINTER(TriPhaseEvents), P]),
         "tri_status_string": (ctypes.c_char_p, [I]),
+        "tri_selftest_bounded_wait": (I, [P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -415,6 +416,14 @@ def tri_compress_step_distance(cache: KvCache, table, slot_pos, opt: TriStepOpti
 def tri_sync_status(status, stream=None) -> int:
     """Wait for the stream, read and clear the device status word; returns the code."""
     return int(library().tri_sync_status(_ptr(status, torch.int32, "status"), _stream(stream)))
+
+
+def tri_selftest_bounded_wait(status, flag=None, stream=None) -> None:
+    """Launch the self-test wait (see the C header): it gives up after the
+    library's wait limit unless ``flag`` (device int32) is non-zero."""
+    fp = None if flag is None else _ptr(flag, torch.int32, "flag")
+    _check(library().tri_selftest_bounded_wait(_ptr(status, torch.int32, "status"), fp, _stream(stream)),
+           "tri_selftest_bounded_wait")
 
 
 def alloc_workspace(cache: KvCache, budget, device=None) -> torch.Tensor:

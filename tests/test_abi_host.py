@@ -47,6 +47,12 @@ def test_status_strings(lib):
 FAKE = 1 << 40           # 16-byte aligned, never dereferenced
 
 
+def test_selftest_wait_rejects_bad_pointers(lib):
+    assert lib.tri_selftest_bounded_wait(None, None, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_selftest_bounded_wait(FAKE + 2, None, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_selftest_bounded_wait(FAKE, FAKE + 1, None) == tri.TRI_ERR_INVALID
+
+
 def _desc(**kw):
     d = dict(L=2, Hkv=8, G=4, D=128, block_size=16, k_pool=FAKE, v_pool=FAKE + 4096, num_blocks=100,
              block_table=FAKE, S=2, max_blocks=50, seq_len=FAKE, cur_pos=FAKE, status=FAKE)

@@ -426,6 +426,30 @@ def test_compress_step_prefix_heavy_units_mix_scratch_and_in_place():
     assert torch.equal(wl.v_pool.view(torch.int16), ev.view(torch.int16))
 
 
+def test_bounded_device_wait_gives_up_and_context_stays_usable():
+    """A device wait that nothing completes ends after the library's wait
+    limit (2 s) with TRI_ERR_TIMEOUT; a flag that is already set ends it at
+    once; and the context then runs a step as usual."""
+    import time
+    status = status_tensor(DEV)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    tri.tri_selftest_bounded_wait(status)                      # barrier nobody arrives at
+    assert tri.tri_sync_status(status) == tri.TRI_ERR_TIMEOUT
+    waited = time.perf_counter() - t0
+    assert 1.5 < waited < 30.0, waited
+    unset = torch.zeros(1, dtype=torch.int32, device=DEV)
+    tri.tri_selftest_bounded_wait(status, unset)               # flag nobody sets
+    assert tri.tri_sync_status(status) == tri.TRI_ERR_TIMEOUT
+    t0 = time.perf_counter()
+    tri.tri_selftest_bounded_wait(status, torch.ones(1, dtype=torch.int32, device=DEV))
+    assert tri.tri_sync_status(status) == tri.TRI_OK
+    assert time.perf_counter() - t0 < 1.0
+    wl = _workload("hkv4", seed=3)
+    out = run_step(wl, gpu_stats(wl), wl.cfg.budget, wl.cfg.window)
+    assert out["status"] == tri.TRI_OK
+
+
 def test_compress_step_replays_from_a_cuda_graph():
     """One step captured in a CUDA graph (its launches with programmatic
     dependencies become graph edges) and replayed on a restored cache gives
