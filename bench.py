@@ -248,7 +248,7 @@ def host_cpu_model():
     return "unknown"
 
 
-def c_oracle_sample(units, stats_fn, deltas, base, budget, window, seconds, threads):
+def c_oracle_sample(units, stats_fn, deltas, base, budget, window, seconds, threads, sinks=0, aggregate="mean"):
     """Time the plain C float64 oracle on units, ``threads`` units at a time
     on the host cores, until about ``seconds`` of wall time have passed.
     Unit inputs are prepared outside the timed region.  Returns (keys
@@ -269,7 +269,7 @@ def c_oracle_sample(units, stats_fn, deltas, base, budget, window, seconds, thre
                 break
             t0 = time.perf_counter()
             list(pool.map(lambda a: compress_unit_c(a[0], a[1], a[2], a[3], a[4], a[5], deltas, base, budget,
-                                                    window), batch))
+                                                    window, sinks, aggregate), batch))
             t_used += time.perf_counter() - t0
             keys_done += sum(a[0].shape[0] for a in batch)
             n += len(batch)
@@ -479,7 +479,10 @@ def run_ours(args, world, rank, local, dist):
     # ---------------------------------------------------- cpu baseline
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens)
+        if distance:
+            cpu = run_cpu_baseline_distance(args, wl, cfg, save_k, save_v, rblocks, lens, max_dist)
+        else:
+            cpu = run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens)
 
     clk = clocks.summary()
     out = {
@@ -638,8 +641,9 @@ def run_e2e(args, tri, cache, wl, qbar, qabs, R, freed, count, save_k, save_v, r
 
 
 def run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens):
-    """The float64 oracle on a bounded sample of this workload's units, on
-    one host core (restored, untouched inputs)."""
+    """The float64 oracle on a bounded sample of this workload's units
+    (restored, untouched inputs): the plain C oracle one unit per host thread
+    on every core, with its one-thread figure and the numpy oracle's beside it."""
     import numpy as np
     import torch
     import oracle
@@ -668,17 +672,11 @@ def run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens):
             yield (unit_rows(wl.k_pool, table[s], n, l, h).cpu(), unit_rows(wl.v_pool, table[s], n, l, h).cpu(),
                    (s, l, h), int(wl.cur_pos[s].item()))
 
-    if args.sinks or args.aggregate != "mean":
-        keys, secs, n = oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
-                                      args.cpu_seconds, args.sinks, args.aggregate)
-        return {"value": round(keys / secs, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
-                "sample": f"{n} random units of this workload ({keys} keys), float64 numpy oracle, 1 thread; "
-                          f"host has {os.cpu_count()} cores", "seconds": round(secs, 2)}
     threads = os.cpu_count() or 1
     keys, secs, n = c_oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
-                                    args.cpu_seconds, threads)
+                                    args.cpu_seconds, threads, args.sinks, args.aggregate)
     c1, cs1, cn1 = c_oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
-                                   min(3.0, args.cpu_seconds), 1)
+                                   min(3.0, args.cpu_seconds), 1, args.sinks, args.aggregate)
     k1, s1, n1 = oracle_sample(units(), stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window,
                                min(4.0, args.cpu_seconds), args.sinks, args.aggregate)
     return {"value": round(keys / secs, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -687,6 +685,58 @@ def run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens):
             "seconds": round(secs, 2), "cpu_model": host_cpu_model(),
             "c_oracle_1_thread": {"value": round(c1 / cs1, 1), "units": cn1, "seconds": round(cs1, 2)},
             "numpy_oracle_1_thread": {"value": round(k1 / s1, 1), "units": n1, "seconds": round(s1, 2)}}
+
+
+def run_cpu_baseline_distance(args, wl, cfg, save_k, save_v, rblocks, lens, max_dist):
+    """The distance-only variant's step in the float64 numpy oracle on units
+    of this workload, one host core: each unit's scores looked up from its
+    (layer, KV head) table, selection, and compaction of rows and positions.
+    The tables of two sampled (layer, KV head) pairs are built once from the
+    oracle's calibration of the query samples and the workload's key centres,
+    outside the timed region (as the device builds its tables once)."""
+    import numpy as np
+    import torch
+    import oracle
+    wl.k_pool[:, rblocks] = save_k
+    wl.v_pool[:, rblocks] = save_v
+    table = wl.block_table.cpu().tolist()
+    rng = np.random.default_rng(1)
+    G = cfg.G
+    pairs = [(int(rng.integers(cfg.L)), int(rng.integers(cfg.Hkv))) for _ in range(2)]
+    tables = {}
+    for l, h in pairs:
+        if wl.q_samples is not None:
+            qb = oracle.calibrate(wl.q_samples[:, l, h * G:(h + 1) * G].double().cpu().numpy())[0]
+        else:
+            qb = wl.qbar[l, h * G:(h + 1) * G].double().cpu().numpy()
+        tables[(l, h)] = oracle.distance_table(qb, wl.key_centres[l, h].double().cpu().numpy(), wl.deltas,
+                                               cfg.base, max_dist, args.aggregate)
+    trig = max(args.trigger, cfg.budget)
+    seqs = [s for s in range(cfg.S) if lens[s] > trig]
+    keys, secs, n = 0, 0.0, 0
+    while seqs and secs < args.cpu_seconds:
+        s = seqs[int(rng.integers(len(seqs)))]
+        l, h = pairs[n % len(pairs)]
+        length, p = lens[s], int(wl.cur_pos[s].item())
+        kb = unit_rows(wl.k_pool, table[s], length, l, h).cpu().view(torch.int16).numpy()
+        vb = unit_rows(wl.v_pool, table[s], length, l, h).cpu().view(torch.int16).numpy()
+        pos = np.arange(length, dtype=np.int64)
+        t0 = time.perf_counter()
+        sc = oracle.distance_scores(tables[(l, h)], p, pos)
+        idx = oracle.select(sc, length, cfg.budget, cfg.window, args.sinks)
+        oracle.compact_rows(kb, idx)
+        oracle.compact_rows(vb, idx)
+        oracle.compact_rows(pos, idx)
+        secs += time.perf_counter() - t0
+        keys += length
+        n += 1
+    if n == 0:
+        return None
+    return {"value": round(keys / secs, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": (f"{n} units of this workload ({keys} keys) on {len(pairs)} (layer, KV head) tables built "
+                       f"once untimed; float64 numpy oracle: table lookup, selection, compaction of rows and "
+                       f"positions, 1 thread; host has {os.cpu_count()} cores"),
+            "seconds": round(secs, 2), "cpu_model": host_cpu_model()}
 
 
 # ---------------------------------------------------------- reference arm

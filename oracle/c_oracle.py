@@ -43,7 +43,7 @@ def _load():
         P, I = ctypes.c_void_p, ctypes.c_int
         lib.tri_oracle_unit.restype = I
         lib.tri_oracle_unit.argtypes = [P, P, I, I, P, P, P, I, ctypes.c_int64, P, I, ctypes.c_double, I, I,
-                                        P, P, P, P]
+                                        I, I, P, P, P, P]
         _lib = lib
     return _lib
 
@@ -53,10 +53,14 @@ def _ptr(a: np.ndarray) -> ctypes.c_void_p:
 
 
 def compress_unit_c(k_bits: np.ndarray, v_bits: np.ndarray, qbar: np.ndarray, qabs: np.ndarray, R: np.ndarray,
-                    p: int, deltas: Sequence[int], base: float, budget: int,
-                    window: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray, np.ndarray]:
+                    p: int, deltas: Sequence[int], base: float, budget: int, window: int, sinks: int = 0,
+                    aggregate: str = "mean") -> Tuple[np.ndarray, np.ndarray, np.ndarray, np.ndarray]:
     """One unit: k_bits / v_bits are bf16 bit patterns [T, D] (int16 or uint16),
-    statistics of its G query heads.  Returns (scores, idx, new K rows, new V rows)."""
+    statistics of its G query heads; ``sinks`` leading slots always kept and
+    the group ``aggregate`` ("mean" or "max") as in the numpy oracle.
+    Returns (scores, idx, new K rows, new V rows)."""
+    if aggregate not in ("mean", "max"):
+        raise ValueError("aggregate must be 'mean' or 'max'")
     lib = _load()
     k = np.ascontiguousarray(k_bits).view(np.uint16)
     v = np.ascontiguousarray(v_bits).view(np.uint16)
@@ -69,8 +73,8 @@ def compress_unit_c(k_bits: np.ndarray, v_bits: np.ndarray, qbar: np.ndarray, qa
     idx = np.empty(max(min(T, budget), 1), dtype=np.int32)
     ko, vo = np.empty_like(k), np.empty_like(v)
     kept = lib.tri_oracle_unit(_ptr(k), _ptr(v), T, D, _ptr(qb), _ptr(qa), _ptr(r), qb.shape[0], int(p), _ptr(d),
-                               d.shape[0], float(base), int(budget), int(window), _ptr(scores), _ptr(idx), _ptr(ko),
-                               _ptr(vo))
+                               d.shape[0], float(base), int(budget), int(window), int(sinks),
+                               1 if aggregate == "max" else 0, _ptr(scores), _ptr(idx), _ptr(ko), _ptr(vo))
     if kept < 0:
         raise ValueError("C oracle rejected its arguments")
     return scores, idx[:kept].astype(np.int64), ko.view(k_bits.dtype), vo.view(v_bits.dtype)

@@ -24,10 +24,11 @@
  *   m_i    = mean_delta exp(j theta_i (p + delta))
  *   c_g,i  = qbar_g,i * m_i
  *   s_g(t) = sum_i Re(c_g,i conj(k_t,i)) + (1 - R_g) sum_i (A_g,i - |qbar_g,i|) |k_t,i|
- *   s(t)   = mean_g s_g(t)
- * Selection: len <= B keeps every slot; otherwise the last W slots and the
- * B - W best of the others by (score descending, slot ascending), output
- * ascending.  Compaction: row j takes row idx_j.
+ *   s(t)   = mean_g s_g(t)   (or max_g s_g(t), the max-over-group variant)
+ * Selection: len <= B keeps every slot; otherwise the first S slots (attention
+ * sinks, a variant; S = 0 for the method), the last W slots and the
+ * B - W - S best of the slots between them by (score descending, slot
+ * ascending), output ascending.  Compaction: row j takes row idx_j.
  */
 #include <math.h>
 #include <stdint.h>
@@ -63,15 +64,18 @@ static int ascending(const void *a, const void *b) {
 
 /*
  * One unit.  keys, vals: bf16 bit patterns [T][D]; qbar [G][D], qabs [G][D/2],
- * R [G] in float64.  Outputs: scores [T], idx [min(T, B)] (returns its
- * length), keys_out / vals_out [T][D] (rows past the kept count unchanged).
- * Returns -1 on a bad argument or allocation failure.
+ * R [G] in float64; sinks: leading slots always kept; agg_max: 0 for the
+ * group mean, 1 for the group maximum.  Outputs: scores [T], idx [min(T, B)]
+ * (returns its length), keys_out / vals_out [T][D] (rows past the kept count
+ * unchanged).  Returns -1 on a bad argument or allocation failure.
  */
 int tri_oracle_unit(const uint16_t *keys, const uint16_t *vals, int T, int D, const double *qbar,
                     const double *qabs, const double *R, int G, int64_t p, const int32_t *deltas, int nd,
-                    double base, int budget, int window, double *scores, int32_t *idx, uint16_t *keys_out,
-                    uint16_t *vals_out) {
-    if (T < 0 || D < 2 || D % 2 || G < 1 || nd < 1 || budget < 1 || window < 0 || window > budget) return -1;
+                    double base, int budget, int window, int sinks, int agg_max, double *scores, int32_t *idx,
+                    uint16_t *keys_out, uint16_t *vals_out) {
+    if (T < 0 || D < 2 || D % 2 || G < 1 || nd < 1 || budget < 1 || window < 0 || sinks < 0 ||
+        window + sinks > budget || (agg_max != 0 && agg_max != 1))
+        return -1;
     const int n = D / 2;
     double *mr = (double *)malloc(sizeof(double) * n * (2 + 3 * G));
     if (!mr) return -1;
@@ -98,9 +102,9 @@ int tri_oracle_unit(const uint16_t *keys, const uint16_t *vals, int T, int D, co
             wt[g * n + i] = (1.0 - R[g]) * (qabs[g * n + i] - sqrt(xr * xr + xi * xi));
         }
     }
-    /* scores: mean over the heads of trig + weighted norm */
+    /* scores: mean (or maximum) over the heads of trig + weighted norm */
     for (int t = 0; t < T; ++t) {
-        double total = 0.0;
+        double total = 0.0, best = 0.0;
         for (int g = 0; g < G; ++g) {
             double trig = 0.0, norm = 0.0;
             for (int i = 0; i < n; ++i) {
@@ -110,9 +114,11 @@ int tri_oracle_unit(const uint16_t *keys, const uint16_t *vals, int T, int D, co
                 trig += cr[g * n + i] * kr + ci[g * n + i] * ki;
                 norm += wt[g * n + i] * sqrt(kr * kr + ki * ki);
             }
-            total += trig + norm;
+            const double sg = trig + norm;
+            total += sg;
+            best = (g == 0 || sg > best) ? sg : best;
         }
-        scores[t] = total / G;
+        scores[t] = agg_max ? best : total / G;
     }
     free(mr);
 
@@ -122,18 +128,19 @@ int tri_oracle_unit(const uint16_t *keys, const uint16_t *vals, int T, int D, co
         kept = T;
         for (int t = 0; t < T; ++t) idx[t] = t;
     } else {
-        const int cand = T - window, take = budget - window;
-        ranked *r = (ranked *)malloc(sizeof(ranked) * (cand > 0 ? cand : 1));
+        const int cand = T - window, take = budget - window - sinks, nr = cand - sinks;
+        ranked *r = (ranked *)malloc(sizeof(ranked) * (nr > 0 ? nr : 1));
         if (!r) return -1;
-        for (int t = 0; t < cand; ++t) {
-            r[t].score = scores[t];
-            r[t].slot = t;
+        for (int t = sinks; t < cand; ++t) {
+            r[t - sinks].score = scores[t];
+            r[t - sinks].slot = t;
         }
-        qsort(r, cand, sizeof(ranked), by_score_then_slot);
-        for (int j = 0; j < take; ++j) idx[j] = r[j].slot;
+        qsort(r, nr, sizeof(ranked), by_score_then_slot);
+        for (int j = 0; j < sinks; ++j) idx[j] = j;
+        for (int j = 0; j < take; ++j) idx[sinks + j] = r[j].slot;
         free(r);
-        qsort(idx, take, sizeof(int32_t), ascending);
-        for (int j = 0; j < window; ++j) idx[take + j] = cand + j;
+        qsort(idx + sinks, take, sizeof(int32_t), ascending);
+        for (int j = 0; j < window; ++j) idx[sinks + take + j] = cand + j;
         kept = budget;
     }
 

@@ -55,3 +55,36 @@ def test_binding_raises_without_the_library(tmp_path):
     r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == "raised True"
+
+
+def _small_cpu_workload():
+    sys.path.insert(0, ROOT)
+    from workload import CONFIGS, make_workload
+    cfg = CONFIGS["l32h8_t32k"].replace(L=2, Hkv=2, G=2, lens=[3000, 900], budget=512, window=64, n_samples=256)
+    wl = make_workload(cfg, device="cpu")
+    rblocks = wl.block_table[:, :32].reshape(-1).long()
+    return cfg, wl, rblocks
+
+
+def _args(**kw):
+    import argparse
+    d = dict(cpu_seconds=0.5, sinks=0, aggregate="mean", trigger=0)
+    d.update(kw)
+    return argparse.Namespace(**d)
+
+
+def test_cpu_baseline_covers_the_variants():
+    """The CPU baseline of a variant bench line times that variant: the C
+    oracle with sinks and the max over the group, and the distance-table step
+    for the distance-only mode."""
+    import bench
+    cfg, wl, rblocks = _small_cpu_workload()
+    save_k, save_v = wl.k_pool[:, rblocks].clone(), wl.v_pool[:, rblocks].clone()
+    lens = wl.seq_len.tolist()
+    for kw in (dict(), dict(sinks=4), dict(aggregate="max")):
+        out = bench.run_cpu_baseline(_args(**kw), wl, cfg, save_k, save_v, rblocks, lens)
+        assert out["kind"] == "oracle" and out["value"] > 0 and out["cores"] >= 1
+        assert out["c_oracle_1_thread"]["value"] > 0 and out["cpu_model"]
+    max_dist = int(wl.cur_pos.max().item()) + 1
+    out = bench.run_cpu_baseline_distance(_args(), wl, cfg, save_k, save_v, rblocks, lens, max_dist)
+    assert out["kind"] == "oracle" and out["value"] > 0 and "table lookup" in out["sample"]

@@ -42,8 +42,34 @@ def test_c_oracle_matches_numpy_oracle(T, G, budget, window):
     assert np.array_equal(k_c, k_py) and np.array_equal(v_c, v_py)
 
 
+@pytest.mark.parametrize("T,G,budget,window,sinks,agg", [(40, 4, 16, 4, 3, "mean"), (200, 2, 64, 8, 5, "max"),
+                                                          (200, 8, 64, 0, 0, "max"), (100, 1, 30, 10, 20, "mean"),
+                                                          (64, 4, 64, 4, 4, "max"), (65, 3, 9, 0, 9, "mean")])
+def test_c_oracle_variants_match_numpy_oracle(T, G, budget, window, sinks, agg):
+    """Attention sinks and the max over the group, as the numpy oracle
+    defines them."""
+    rng = np.random.default_rng(T * 13 + G + sinks)
+    D, p, base = 128, T + 5, 1e6
+    deltas = [1, 2, 4, 8, 1024]
+    kb, vb, qbar, qabs, R = _unit(rng, T, D, G, dup=True)
+    s_c, idx_c, k_c, v_c = compress_unit_c(kb, vb, qbar, qabs, R, p, deltas, base, budget, window, sinks, agg)
+    kf = torch.from_numpy(kb).view(torch.bfloat16).double().numpy()
+    s_py, idx_py, k_py, v_py = oracle.compress_unit(kf, kb, vb, qbar, qabs, R, p, deltas, base, budget, window,
+                                                    sinks=sinks, aggregate=agg)
+    scale = max(1.0, float(np.max(np.abs(s_py))))
+    np.testing.assert_allclose(s_c, s_py, rtol=1e-12, atol=1e-12 * scale)
+    assert np.array_equal(idx_c, idx_py)
+    if T > budget:
+        assert np.array_equal(idx_c[:sinks], np.arange(sinks))
+    assert np.array_equal(k_c, k_py) and np.array_equal(v_c, v_py)
+
+
 def test_c_oracle_rejects_bad_arguments():
     rng = np.random.default_rng(0)
     kb, vb, qbar, qabs, R = _unit(rng, 10, 128, 1)
     with pytest.raises(ValueError):
         compress_unit_c(kb, vb, qbar, qabs, R, 10, [1], 1e4, 4, 5)        # window > budget
+    with pytest.raises(ValueError):
+        compress_unit_c(kb, vb, qbar, qabs, R, 10, [1], 1e4, 4, 2, 3)     # sinks + window > budget
+    with pytest.raises(ValueError):
+        compress_unit_c(kb, vb, qbar, qabs, R, 10, [1], 1e4, 4, 2, 0, "median")
