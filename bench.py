@@ -687,6 +687,37 @@ def run_cpu_baseline(args, wl, cfg, save_k, save_v, rblocks, lens):
             "numpy_oracle_1_thread": {"value": round(k1 / s1, 1), "units": n1, "seconds": round(s1, 2)}}
 
 
+def distance_oracle_sample(wl, cfg, lens, tables, pairs, seconds, sinks, trigger, rng):
+    """Time the numpy oracle's distance-table step (lookup, selection,
+    compaction of rows and positions) on units of the compressed sequences,
+    cycling over the (layer, KV head) pairs whose tables are given, until
+    about ``seconds`` have passed.  Returns (keys, seconds, units)."""
+    import numpy as np
+    import torch
+    import oracle
+    table = wl.block_table.cpu().tolist()
+    trig = max(trigger, cfg.budget)
+    seqs = [s for s in range(cfg.S) if lens[s] > trig]
+    keys, secs, n = 0, 0.0, 0
+    while seqs and secs < seconds:
+        s = seqs[int(rng.integers(len(seqs)))]
+        l, h = pairs[n % len(pairs)]
+        length, p = lens[s], int(wl.cur_pos[s].item())
+        kb = unit_rows(wl.k_pool, table[s], length, l, h).cpu().view(torch.int16).numpy()
+        vb = unit_rows(wl.v_pool, table[s], length, l, h).cpu().view(torch.int16).numpy()
+        pos = np.arange(length, dtype=np.int64)
+        t0 = time.perf_counter()
+        sc = oracle.distance_scores(tables[(l, h)], p, pos)
+        idx = oracle.select(sc, length, cfg.budget, cfg.window, sinks)
+        oracle.compact_rows(kb, idx)
+        oracle.compact_rows(vb, idx)
+        oracle.compact_rows(pos, idx)
+        secs += time.perf_counter() - t0
+        keys += length
+        n += 1
+    return keys, secs, n
+
+
 def run_cpu_baseline_distance(args, wl, cfg, save_k, save_v, rblocks, lens, max_dist):
     """The distance-only variant's step in the float64 numpy oracle on units
     of this workload, one host core: each unit's scores looked up from its
@@ -699,7 +730,6 @@ def run_cpu_baseline_distance(args, wl, cfg, save_k, save_v, rblocks, lens, max_
     import oracle
     wl.k_pool[:, rblocks] = save_k
     wl.v_pool[:, rblocks] = save_v
-    table = wl.block_table.cpu().tolist()
     rng = np.random.default_rng(1)
     G = cfg.G
     pairs = [(int(rng.integers(cfg.L)), int(rng.integers(cfg.Hkv))) for _ in range(2)]
@@ -711,25 +741,8 @@ def run_cpu_baseline_distance(args, wl, cfg, save_k, save_v, rblocks, lens, max_
             qb = wl.qbar[l, h * G:(h + 1) * G].double().cpu().numpy()
         tables[(l, h)] = oracle.distance_table(qb, wl.key_centres[l, h].double().cpu().numpy(), wl.deltas,
                                                cfg.base, max_dist, args.aggregate)
-    trig = max(args.trigger, cfg.budget)
-    seqs = [s for s in range(cfg.S) if lens[s] > trig]
-    keys, secs, n = 0, 0.0, 0
-    while seqs and secs < args.cpu_seconds:
-        s = seqs[int(rng.integers(len(seqs)))]
-        l, h = pairs[n % len(pairs)]
-        length, p = lens[s], int(wl.cur_pos[s].item())
-        kb = unit_rows(wl.k_pool, table[s], length, l, h).cpu().view(torch.int16).numpy()
-        vb = unit_rows(wl.v_pool, table[s], length, l, h).cpu().view(torch.int16).numpy()
-        pos = np.arange(length, dtype=np.int64)
-        t0 = time.perf_counter()
-        sc = oracle.distance_scores(tables[(l, h)], p, pos)
-        idx = oracle.select(sc, length, cfg.budget, cfg.window, args.sinks)
-        oracle.compact_rows(kb, idx)
-        oracle.compact_rows(vb, idx)
-        oracle.compact_rows(pos, idx)
-        secs += time.perf_counter() - t0
-        keys += length
-        n += 1
+    keys, secs, n = distance_oracle_sample(wl, cfg, lens, tables, pairs, args.cpu_seconds, args.sinks,
+                                           args.trigger, rng)
     if n == 0:
         return None
     return {"value": round(keys / secs, 1), "unit": UNIT, "cores": 1, "kind": "oracle",
@@ -779,14 +792,22 @@ def run_reference(args, world, rank):
         return stats[0][0, h * G:(h + 1) * G], stats[1][0, h * G:(h + 1) * G], stats[2][0, h * G:(h + 1) * G]
 
     it = units()
-    plain = not args.sinks and args.aggregate == "mean"
-    threads = (os.cpu_count() or 1) if plain else 1
+    threads = os.cpu_count() or 1
+    distance = args.score_mode == "distance"
+    if distance:
+        # the distance-only variant: tables of two KV heads, built once untimed
+        threads = 1
+        pairs = [(0, h) for h in range(min(2, cfg.Hkv))]
+        max_dist = int(wl.cur_pos.max().item()) + 1
+        tables = {(l, h): oracle.distance_table(stats_fn(l, h)[0], wl.key_centres[l, h].double().numpy(),
+                                                wl.deltas, cfg.base, max_dist, args.aggregate) for l, h in pairs}
+        drng = np.random.default_rng(1)
 
     def sample_once(seconds):
-        if plain:
-            return c_oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, seconds, threads)
-        return oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, seconds, args.sinks,
-                             args.aggregate)
+        if distance:
+            return distance_oracle_sample(wl, cfg, lens, tables, pairs, seconds, args.sinks, args.trigger, drng)
+        return c_oracle_sample(it, stats_fn, wl.deltas, cfg.base, cfg.budget, cfg.window, seconds, threads,
+                               args.sinks, args.aggregate)
 
     for _ in range(args.warmup):
         sample_once(0.0)
@@ -798,14 +819,16 @@ def run_reference(args, world, rank):
         secs += s_
         n_units += n
     value = keys / secs
-    kind = (f"plain C float64 oracle, one unit per host thread on {threads} threads" if plain
-            else "float64 numpy oracle, 1 thread")
+    kind = ("float64 numpy oracle, distance-table lookup, selection and compaction, 1 thread (tables of "
+            f"{len(pairs)} KV heads built once, untimed)" if distance else
+            f"plain C float64 oracle, one unit per host thread on {threads} threads")
     sample = f"{n_units} units of the {cfg.name} workload shape over {args.steps} steps, {kind}"
     out = {"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * secs / args.steps, 3),
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "config": {"workload": cfg.name, "L": cfg.L, "Hkv": cfg.Hkv, "G": cfg.G, "D": 128,
-                      "seq_lens": cfg.lens, "budget": cfg.budget, "window": cfg.window},
+                      "seq_lens": cfg.lens, "budget": cfg.budget, "window": cfg.window, "sinks": args.sinks,
+                      "aggregate": args.aggregate, "score_mode": args.score_mode},
            "cpu_baseline": {"value": round(value, 1), "unit": UNIT, "cores": threads, "kind": "oracle",
                             "sample": sample, "cpu_model": host_cpu_model()},
            "e2e": {"value": round(value, 1), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

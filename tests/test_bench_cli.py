@@ -88,3 +88,17 @@ def test_cpu_baseline_covers_the_variants():
     max_dist = int(wl.cur_pos.max().item()) + 1
     out = bench.run_cpu_baseline_distance(_args(), wl, cfg, save_k, save_v, rblocks, lens, max_dist)
     assert out["kind"] == "oracle" and out["value"] > 0 and "table lookup" in out["sample"]
+
+
+def test_reference_arm_times_the_requested_variant():
+    for extra, marker in ((["--aggregate", "max", "--sinks", "2"], "plain C float64 oracle"),
+                          (["--score-mode", "distance"], "distance-table lookup")):
+        r = _run(["--impl", "reference", "--workload", "head1_t4096", "--steps", "1", "--warmup", "0",
+                  "--cpu-seconds", "1"] + extra)
+        assert r.returncode == 0, r.stderr[-2000:]
+        d = json.loads(r.stdout.strip().splitlines()[-1])
+        assert d["value"] > 0 and marker in d["cpu_baseline"]["sample"]
+        if "--aggregate" in extra:
+            assert d["config"]["aggregate"] == "max" and d["config"]["sinks"] == 2
+        else:
+            assert d["config"]["score_mode"] == "distance"
