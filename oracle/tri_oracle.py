@@ -232,10 +232,16 @@ def freed_blocks(table_row: Sequence[int], old_len: int, kept: int, block_size: 
 
 # ----------------------------------------------------------------------------
 # Paged cache plumbing (layout [L][num_blocks][Hkv][block_size][D])
+# [GeoTrick] "Solving the Memory Fragmentation Problem" and "Why Existing KV
+# Cache Compression Breaks in Production": a sequence's cache is a chain of
+# fixed-size pages; its block table names the page of every run of
+# block_size slots, so slot t sits in row t mod block_size of page
+# table[t div block_size].
 # ----------------------------------------------------------------------------
 
 def unit_rows(pool: np.ndarray, table_row: Sequence[int], length: int, l: int, h: int) -> np.ndarray:
-    """The ``length`` cached rows of (layer l, KV head h) of one sequence."""
+    """The ``length`` cached rows of (layer l, KV head h) of one sequence:
+    row t is pool[l, table_row[t // bs], h, t % bs]."""
     bs = pool.shape[3]
     out = np.empty((length, pool.shape[4]), dtype=pool.dtype)
     for t in range(length):
@@ -244,6 +250,7 @@ def unit_rows(pool: np.ndarray, table_row: Sequence[int], length: int, l: int, h
 
 
 def store_unit_rows(pool: np.ndarray, table_row: Sequence[int], rows: np.ndarray, l: int, h: int) -> None:
+    """Write rows[t] to pool[l, table_row[t // bs], h, t % bs] for every t."""
     bs = pool.shape[3]
     for t in range(rows.shape[0]):
         pool[l, int(table_row[t // bs]), h, t % bs] = rows[t]

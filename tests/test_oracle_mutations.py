@@ -197,6 +197,26 @@ def _calibrate_rms(q):
     return T.from_bands(zbar), A, np.where(den > 0, num / np.where(den > 0, den, 1), 1.0)
 
 
+def _unit_rows_table_ignored(pool, table_row, length, l, h):
+    bs = pool.shape[3]
+    return np.stack([pool[l, t // bs, h, t % bs] for t in range(length)]) if length else \
+        np.empty((0, pool.shape[4]), pool.dtype)
+
+
+def _unit_rows_div_mod_swapped(pool, table_row, length, l, h):
+    bs = pool.shape[3]
+    out = np.empty((length, pool.shape[4]), dtype=pool.dtype)
+    for t in range(length):
+        out[t] = pool[l, int(table_row[t % bs]), h, t // bs]
+    return out
+
+
+def _store_unit_rows_div_mod_swapped(pool, table_row, rows, l, h):
+    bs = pool.shape[3]
+    for t in range(rows.shape[0]):
+        pool[l, int(table_row[t % bs]), h, t // bs] = rows[t]
+
+
 MUTATIONS = [
     ("future_phase_mean", _phase_sign_flipped),
     ("future_phase_mean", _phase_summed),
@@ -220,6 +240,9 @@ MUTATIONS = [
     ("freed_blocks", _freed_floor),
     ("calibrate", _calibrate_vector_norms),
     ("calibrate", _calibrate_rms),
+    ("unit_rows", _unit_rows_table_ignored),
+    ("unit_rows", _unit_rows_div_mod_swapped),
+    ("store_unit_rows", _store_unit_rows_div_mod_swapped),
 ]
 
 

@@ -415,6 +415,60 @@ def test_freed_blocks_are_the_emptied_tail():
             assert len(f) == -(-length // 16) - (-(-kept // 16))
 
 
+def _identity_pool(L, NB, Hkv, bs):
+    """A pool whose row [l, b, h, r] holds its own address (l, b, h, r)."""
+    pool = np.zeros((L, NB, Hkv, bs, 4), dtype=np.int64)
+    for l, b, h, r in itertools.product(range(L), range(NB), range(Hkv), range(bs)):
+        pool[l, b, h, r] = (l, b, h, r)
+    return pool
+
+
+def test_unit_rows_follow_the_block_table():
+    """Slot t of a unit lives in row t mod 16 of the table's block t div 16
+    ([GeoTrick] "Solving the Memory Fragmentation Problem": a sequence's
+    cache is a chain of fixed-size pages named by its block table).  Block
+    size 4 here; every expected address is written out by hand."""
+    pool = _identity_pool(L=2, NB=8, Hkv=3, bs=4)
+    table_row = [5, 2, 7, 0]                       # a permuted table
+    rows = oracle.unit_rows(pool, table_row, 14, 1, 2)
+    assert rows.shape == (14, 4)
+    expected = {
+        0: (1, 5, 2, 0), 1: (1, 5, 2, 1), 3: (1, 5, 2, 3),     # block table_row[0] = 5
+        4: (1, 2, 2, 0), 6: (1, 2, 2, 2),                      # block table_row[1] = 2
+        8: (1, 7, 2, 0), 9: (1, 7, 2, 1), 11: (1, 7, 2, 3),    # block table_row[2] = 7
+        12: (1, 0, 2, 0), 13: (1, 0, 2, 1),                    # block table_row[3] = 0
+    }
+    for t, addr in expected.items():
+        assert tuple(rows[t]) == addr, t
+    # another layer and head through the same table
+    rows0 = oracle.unit_rows(pool, table_row, 6, 0, 0)
+    assert [tuple(r) for r in rows0] == [(0, 5, 0, 0), (0, 5, 0, 1), (0, 5, 0, 2), (0, 5, 0, 3),
+                                         (0, 2, 0, 0), (0, 2, 0, 1)]
+    assert oracle.unit_rows(pool, table_row, 0, 1, 1).shape == (0, 4)
+
+
+def test_store_unit_rows_writes_exactly_the_table_addresses():
+    """Storing a unit's rows touches rows (l, table[t div 16], h, t mod 16)
+    for t < len and nothing else (block size 4 here, addresses by hand)."""
+    L, NB, Hkv, bs = 2, 8, 3, 4
+    pool = _identity_pool(L, NB, Hkv, bs)
+    before = pool.copy()
+    table_row = [6, 1, 4]
+    marks = np.full((10, 4), -1, dtype=np.int64)
+    marks[:, 0] = np.arange(10)
+    oracle.tri_oracle.store_unit_rows(pool, table_row, marks, 0, 1)
+    written = {(0, 6, 1, 0): 0, (0, 6, 1, 1): 1, (0, 6, 1, 2): 2, (0, 6, 1, 3): 3,
+               (0, 1, 1, 0): 4, (0, 1, 1, 1): 5, (0, 1, 1, 2): 6, (0, 1, 1, 3): 7,
+               (0, 4, 1, 0): 8, (0, 4, 1, 1): 9}
+    for addr in itertools.product(range(L), range(NB), range(Hkv), range(bs)):
+        if addr in written:
+            assert pool[addr][0] == written[addr] and pool[addr][1] == -1, addr
+        else:
+            np.testing.assert_array_equal(pool[addr], before[addr])
+    # reading back through the table returns what was stored
+    np.testing.assert_array_equal(oracle.unit_rows(pool, table_row, 10, 0, 1), marks)
+
+
 def test_paged_step_equals_unit_by_unit():
     """The paged compress_step moves exactly what compress_unit says, per unit,
     and leaves other rows alone."""
