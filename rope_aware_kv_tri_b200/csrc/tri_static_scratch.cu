@@ -10,9 +10,18 @@
 // The array lives at file scope below.  Every GPU that loads this library
 // holds it (TRI_STATIC_SCRATCH_BYTES) until the process exits.  Host code
 // cannot use the array's name as a device address, so the address is looked
-// up with cudaGetSymbolAddress once per device, with that device current,
-// on the first call made there, and cached.
+// up with cudaGetSymbolAddress, with the device current, and cached.
+//
+// The array belongs to the CUDA context the library's module is loaded in:
+// if that context is destroyed (cudaDeviceReset, or a reset of the device's
+// primary context by any other code in the process) a new context holds a
+// new copy of the array, possibly at another address.  The cache is
+// therefore keyed by the unique id of the current context (cuCtxGetId), not
+// by the device ordinal: a call made in a context other than the one the
+// cached address came from looks the address up again.
 #include <mutex>
+
+#include <cuda.h>
 
 #include "tri_attention.h"
 
@@ -21,25 +30,79 @@ namespace {
 static __device__ __align__(256) unsigned char g_scratch[TRI_STATIC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 128;
-std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {nullptr};
 
-// Device address of g_scratch on the current device (first call per device
-// performs the lookup).
-tri_status scratch_on_current_device(void** out) {
+struct CachedAddress {
+    unsigned long long ctx_id;   // unique id of the context the address belongs to (0: none)
+    void* addr;
+};
+
+std::mutex g_mu;
+CachedAddress g_cache[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Driver entry points that name the current context (looked up once).
+bool context_entry_points(CtxGetCurrentFn& get_current, CtxGetIdFn& get_id) {
+    static CtxGetCurrentFn s_current = nullptr;
+    static CtxGetIdFn s_id = nullptr;
+    static bool tried = false;
+    if (!tried) {   // called with g_mu held
+        tried = true;
+        void* a = nullptr;
+        void* b = nullptr;
+        cudaDriverEntryPointQueryResult qa, qb;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+            qa == cudaDriverEntryPointSuccess &&
+            cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+            qb == cudaDriverEntryPointSuccess) {
+            s_current = reinterpret_cast<CtxGetCurrentFn>(a);
+            s_id = reinterpret_cast<CtxGetIdFn>(b);
+        }
+    }
+    get_current = s_current;
+    get_id = s_id;
+    return s_current != nullptr && s_id != nullptr;
+}
+
+// Unique id of the calling thread's current context; false if there is none
+// or it cannot be named (then nothing is cached).
+bool current_context_id(unsigned long long& id) {
+    CtxGetCurrentFn get_current;
+    CtxGetIdFn get_id;
+    if (!context_entry_points(get_current, get_id)) return false;
+    CUcontext ctx = nullptr;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return false;
+    return get_id(ctx, &id) == CUDA_SUCCESS && id != 0;
+}
+
+// Device address of g_scratch in the current context.
+tri_status scratch_in_current_context(void** out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TRI_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_mu);
-    if (g_scratch_addr[dev] == nullptr) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return TRI_ERR_CUDA;
-        g_scratch_addr[dev] = p;
+    unsigned long long id = 0;
+    if (current_context_id(id) && g_cache[dev].ctx_id == id && g_cache[dev].addr != nullptr) {
+        *out = g_cache[dev].addr;
+        return TRI_OK;
     }
-    *out = g_scratch_addr[dev];
+    void* p = nullptr;
+    // The lookup makes the device's context current if no context was yet.
+    if (cudaGetSymbolAddress(&p, g_scratch) != cudaSuccess || p == nullptr) return TRI_ERR_CUDA;
+    if (current_context_id(id)) {
+        g_cache[dev].ctx_id = id;
+        g_cache[dev].addr = p;
+    } else {
+        g_cache[dev].ctx_id = 0;    // cannot tell contexts apart: look up on every call
+        g_cache[dev].addr = nullptr;
+    }
+    *out = p;
     return TRI_OK;
 }
 
 }  // namespace
+
+extern "C" size_t tri_static_scratch_bytes(void) { return (size_t)TRI_STATIC_SCRATCH_BYTES; }
 
 extern "C" tri_status tri_compress_step_static_scratch(tri_kv_desc* desc, const float* qbar, const float* qabs,
                                                        const float* R, double rope_base, const int32_t* deltas,
@@ -50,10 +113,11 @@ extern "C" tri_status tri_compress_step_static_scratch(tri_kv_desc* desc, const 
     if (need > (size_t)TRI_STATIC_SCRATCH_BYTES) return TRI_ERR_UNSUPPORTED;
     void* ws = nullptr;
     if (need > 0) {
-        const tri_status st = scratch_on_current_device(&ws);
+        const tri_status st = scratch_in_current_context(&ws);
         if (st != TRI_OK) return st;
     }
-    // need == 0 means the descriptor is invalid: tri_compress_step reports why.
+    // need == 0 means the descriptor or the budget is invalid:
+    // tri_compress_step reports why before touching the workspace.
     return tri_compress_step(desc, qbar, qabs, R, rope_base, deltas, n_deltas, budget, window, freed_ids,
                              freed_count, idx_out, ws, (size_t)TRI_STATIC_SCRATCH_BYTES, nullptr, stream);
 }

@@ -11,7 +11,10 @@ These tests call that entry point through the C ABI and check that, on two
 calls in a row with different caches (so the second call starts from the
 scratch contents the first one left behind), it produces exactly what
 tri_compress_step with a caller workspace produces: the same kept slots,
-bit-identical K/V pools, the same freed blocks and lengths.  The file is
+bit-identical K/V pools, the same freed blocks and lengths; that further
+calls leave the device's free memory and torch's allocated bytes unchanged;
+and that shapes beyond the array, an invalid descriptor and a budget above
+the library's maximum are refused before anything is launched.  The file is
 named so that pytest collects it last.
 """
 
@@ -60,7 +63,7 @@ def test_static_scratch_matches_workspace_entry_on_two_calls_in_a_row():
     for seed, cfg in enumerate(CASES):
         a = make_workload(cfg, device=DEV, seed=seed)        # for the static-scratch call
         b = make_workload(cfg, device=DEV, seed=seed)        # identical copy for the workspace call
-        assert tri.tri_workspace_size(cache_of(a), cfg.budget) <= tri.TRI_STATIC_SCRATCH_BYTES
+        assert tri.tri_workspace_size(cache_of(a), cfg.budget) <= tri.tri_static_scratch_bytes()
         stats = gpu_stats(a)
         got = _run(a, stats, static=True)
         want = _run(b, stats, static=False)
@@ -78,7 +81,7 @@ def test_static_scratch_rejects_shapes_beyond_its_size():
     table = torch.zeros(1, max_blocks, dtype=torch.int32, device=DEV)
     cache = tri.KvCache(k, k.clone(), table, torch.zeros(1, dtype=torch.int32, device=DEV),
                         torch.zeros(1, dtype=torch.int64, device=DEV), torch.zeros(1, dtype=torch.int32, device=DEV), 4)
-    assert tri.tri_workspace_size(cache, 64) > tri.TRI_STATIC_SCRATCH_BYTES
+    assert tri.tri_workspace_size(cache, 64) > tri.tri_static_scratch_bytes()
     st = (torch.zeros(L, Hkv * 4, 128, device=DEV), torch.zeros(L, Hkv * 4, 64, device=DEV),
           torch.ones(L, Hkv * 4, device=DEV))
     freed = torch.empty(max_blocks, dtype=torch.int32, device=DEV)
@@ -86,3 +89,58 @@ def test_static_scratch_rejects_shapes_beyond_its_size():
     with pytest.raises(tri.TriError) as e:
         tri.tri_compress_step_static_scratch(cache, *st, 1e4, [1], 64, 8, freed, count)
     assert e.value.code == tri.TRI_ERR_UNSUPPORTED
+
+
+def _small_cache_and_outputs(seed):
+    cfg = CASES[1]
+    wl = make_workload(cfg, device=DEV, seed=seed)
+    freed = torch.empty(cfg.S * wl.max_blocks, dtype=torch.int32, device=DEV)
+    count = torch.empty(1, dtype=torch.int32, device=DEV)
+    return wl, cache_of(wl), freed, count
+
+
+def test_static_scratch_calls_allocate_nothing():
+    wl, cache, freed, count = _small_cache_and_outputs(5)
+    cfg = wl.cfg
+    stats = gpu_stats(wl)
+    save = (wl.k_pool.clone(), wl.v_pool.clone(), wl.seq_len.clone())
+
+    def call():
+        wl.k_pool.copy_(save[0])
+        wl.v_pool.copy_(save[1])
+        wl.seq_len.copy_(save[2])
+        tri.tri_compress_step_static_scratch(cache, *stats, cfg.base, wl.deltas, cfg.budget, cfg.window,
+                                             freed, count)
+
+    call()                                   # warm-up: module load, symbol lookup
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for _ in range(3):
+        tri.tri_compress_step_static_scratch(cache, *stats, cfg.base, wl.deltas, cfg.budget, cfg.window,
+                                             freed, count)
+    torch.cuda.synchronize()
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0, f"device free memory changed by {free0 - free1} bytes"
+
+
+def test_static_scratch_refuses_invalid_descriptor_and_budget():
+    wl, cache, freed, count = _small_cache_and_outputs(6)
+    cfg = wl.cfg
+    stats = gpu_stats(wl)
+    before = (wl.k_pool.clone(), wl.seq_len.clone())
+    bad = tri.KvCache(wl.k_pool, wl.v_pool, wl.block_table, wl.seq_len, wl.cur_pos, cache.status, cfg.G)
+    bad.desc.L = 0                                           # no layers: invalid descriptor
+    with pytest.raises(tri.TriError) as e:
+        tri.tri_compress_step_static_scratch(bad, *stats, cfg.base, wl.deltas, cfg.budget, cfg.window, freed, count)
+    assert e.value.code == tri.TRI_ERR_INVALID
+    with pytest.raises(tri.TriError) as e:
+        tri.tri_compress_step_static_scratch(cache, *stats, cfg.base, wl.deltas, tri.TRI_MAX_BUDGET + 1,
+                                             cfg.window, freed, count)
+    assert e.value.code == tri.TRI_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.equal(wl.k_pool.view(torch.int16), before[0].view(torch.int16))
+    assert torch.equal(wl.seq_len, before[1])
