@@ -258,9 +258,14 @@ tri_status tri_compress_step(tri_kv_desc *desc, const float *qbar, const float *
  *   - Shapes whose tri_workspace_size(desc, budget) exceeds
  *     TRI_STATIC_SCRATCH_BYTES are rejected with TRI_ERR_UNSUPPORTED before
  *     anything is launched (use tri_compress_step with a workspace instead).
- *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current and caches it; make
- *     that first call before capturing the stream into a CUDA graph.
+ *   - The first call in a CUDA context looks up the array's device address
+ *     (cudaGetSymbolAddress) with that context current and caches it, keyed
+ *     by the context's unique id; make that first call before capturing the
+ *     stream into a CUDA graph.  The array belongs to the context: after
+ *     cudaDeviceReset (or anything else that destroys the device's context)
+ *     the next call runs in a new context, holding a new copy of the array,
+ *     and looks the address up again, so no call ever uses an address of a
+ *     destroyed context.  Nothing of an earlier context's scratch survives.
  *   - All calls share the one array and it keeps the last call's contents.
  *     Every call rewrites all of the scratch it reads, so nothing in it needs
  *     to start at zero; but two calls whose work overlaps on the GPU (other
@@ -271,6 +276,9 @@ tri_status tri_compress_step(tri_kv_desc *desc, const float *qbar, const float *
  * phase events).
  */
 #define TRI_STATIC_SCRATCH_BYTES (16u << 20)
+/* The size of that array as built into this library (TRI_STATIC_SCRATCH_BYTES
+ * of the header it was compiled with); a host-only query, no CUDA call. */
+size_t tri_static_scratch_bytes(void);
 tri_status tri_compress_step_static_scratch(tri_kv_desc *desc, const float *qbar, const float *qabs,
                                             const float *R, double rope_base, const int32_t *deltas,
                                             int n_deltas, int budget, int window, int32_t *freed_ids,
@@ -303,6 +311,13 @@ tri_status tri_compress_step_static_scratch(tri_kv_desc *desc, const float *qbar
  *               query (what tri_build_query computes).  TRI_AGG_MAX: their
  *               maximum, each head scored on its own; G must be 1, 2, 4 or 8
  *               (TRI_ERR_UNSUPPORTED otherwise).
+ *   check_stats : non-zero: tri_compress_step_ex first runs the checks of
+ *               tri_check_stats on the statistics it is given; if any head
+ *               fails them (NONFINITE, R_RANGE or NORM_WEIGHT below), it
+ *               raises TRI_DEVFLAG_STATS and changes nothing: no row moves,
+ *               seq_len, the free list and idx_out are left as they are and
+ *               *freed_count = 0.  Costs one small extra launch.  Ignored by
+ *               the selection-only and distance-table entry points.
  * ---------------------------------------------------------------------- */
 #define TRI_AGG_MEAN 0
 #define TRI_AGG_MAX  1
@@ -313,6 +328,7 @@ typedef struct {
     int sinks;
     int trigger;
     int aggregate;
+    int check_stats;
 } tri_step_options;
 
 /*
@@ -334,6 +350,41 @@ typedef struct {
  * room (push); that call changed neither the list nor the block table. */
 #define TRI_DEVFLAG_FREELIST   8
 #define TRI_ERR_FREELIST       8  /* tri_sync_status: TRI_DEVFLAG_FREELIST */
+
+/*
+ * tri_check_stats - check head statistics before a step uses them ([Review]
+ * "Calibration statistics are tied to a specific model": statistics of
+ * another model, or a damaged statistics file, raise no error by
+ * themselves; the step only keeps the wrong keys).  For every one of the
+ * n = L*Hq heads (qbar [L][Hq][D], qabs [L][Hq][D/2], R [L][Hq], as for
+ * tri_build_query) it checks what any valid statistics satisfy:
+ *   TRI_STATS_NONFINITE   a NaN or infinity in the head's qbar, qabs or R;
+ *   TRI_STATS_R_RANGE     R outside [0, 1];
+ *   TRI_STATS_NORM_WEIGHT qabs_i < |qbar_i| for some band beyond a relative
+ *                         1e-5 (a mean of magnitudes is never below the
+ *                         magnitude of the mean; a negative norm weight
+ *                         (1 - R)(qabs_i - |qbar_i|) inverts the ranking);
+ * and reports, without treating it as a failure,
+ *   TRI_STATS_R_MISMATCH  R differs from sum_i |qbar_i| / sum_i qabs_i (the
+ *                         concentration tri_calibrate_centers computes) by
+ *                         more than 1e-3 relative.
+ *   head_flags : NULL, or int32 [L][Hq] out: the bits above per head
+ *   status     : device status word; TRI_DEVFLAG_STATS is OR-ed into it if
+ *                any head has NONFINITE, R_RANGE or NORM_WEIGHT
+ * Errors: TRI_ERR_INVALID (null or misaligned pointer, L or Hq < 1, size
+ * overflow), TRI_ERR_UNSUPPORTED (D != 128), TRI_ERR_CUDA.  Asynchronous:
+ * tri_sync_status() returns TRI_ERR_STATS when the flag was raised.
+ */
+#define TRI_STATS_NONFINITE    1
+#define TRI_STATS_R_RANGE      2
+#define TRI_STATS_NORM_WEIGHT  4
+#define TRI_STATS_R_MISMATCH   8
+/* Device status bit: statistics failed the check (tri_check_stats, or a step
+ * run with check_stats, which then changed nothing). */
+#define TRI_DEVFLAG_STATS      16
+#define TRI_ERR_STATS          9  /* tri_sync_status: TRI_DEVFLAG_STATS */
+tri_status tri_check_stats(const float *qbar, const float *qabs, const float *R, int L, int Hq, int D,
+                           int32_t *head_flags, int32_t *status, cudaStream_t stream);
 
 /* Workspace bytes of tri_score_ex / tri_compress_step_ex with these options
  * (TRI_AGG_MAX keeps G coefficient sets per unit).  0 if invalid. */
@@ -474,7 +525,8 @@ tri_status tri_compress_step_distance(tri_kv_desc *desc, const float *table, int
 /*
  * tri_sync_status - wait for `stream`, read the device status word, clear it,
  * and return TRI_OK or the error its bits name (BOUNDS before TIMEOUT before
- * FREELIST before NONFINITE).  TRI_ERR_CUDA if the stream itself reports an error.
+ * FREELIST before STATS before NONFINITE).  TRI_ERR_CUDA if the stream itself
+ * reports an error.
  */
 tri_status tri_sync_status(int32_t *status, cudaStream_t stream);
 

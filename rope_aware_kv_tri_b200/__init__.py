@@ -29,6 +29,13 @@ TRI_ERR_TIMEOUT = 5
 TRI_ERR_NONFINITE = 6
 TRI_ERR_WORKSPACE = 7
 TRI_ERR_FREELIST = 8
+TRI_ERR_STATS = 9
+
+TRI_DEVFLAG_STATS = 16
+TRI_STATS_NONFINITE = 1
+TRI_STATS_R_RANGE = 2
+TRI_STATS_NORM_WEIGHT = 4
+TRI_STATS_R_MISMATCH = 8
 
 TRI_AGG_MEAN = 0
 TRI_AGG_MAX = 1
@@ -44,9 +51,9 @@ EXPORTS = (
     "tri_select_topk", "tri_compact_kv", "tri_compress_step", "tri_compress_step_static_scratch",
     "tri_sync_status", "tri_status_string", "tri_workspace_size_ex", "tri_score_ex", "tri_select_topk_ex",
     "tri_compress_step_ex", "tri_reserve_blocks", "tri_distance_table", "tri_score_distance",
-    "tri_compress_step_distance", "tri_selftest_bounded_wait",
+    "tri_compress_step_distance", "tri_selftest_bounded_wait", "tri_static_scratch_bytes",
+    "tri_check_stats",
 )
-TRI_STATIC_SCRATCH_BYTES = 16 << 20
 
 
 class TriError(RuntimeError):
@@ -80,7 +87,7 @@ class TriStepOptions(ctypes.Structure):
     """Mirror of ``tri_step_options``."""
 
     _fields_ = [("budget", ctypes.c_int), ("window", ctypes.c_int), ("sinks", ctypes.c_int),
-                ("trigger", ctypes.c_int), ("aggregate", ctypes.c_int)]
+                ("trigger", ctypes.c_int), ("aggregate", ctypes.c_int), ("check_stats", ctypes.c_int)]
 
 
 class TriFreeList(ctypes.Structure):
@@ -119,8 +126,8 @@ class FreeList:
 
 
 def step_options(budget: int, window: int, sinks: int = 0, trigger: int = 0,
-                 aggregate: int = TRI_AGG_MEAN) -> TriStepOptions:
-    return TriStepOptions(int(budget), int(window), int(sinks), int(trigger), int(aggregate))
+                 aggregate: int = TRI_AGG_MEAN, check_stats: bool = False) -> TriStepOptions:
+    return TriStepOptions(int(budget), int(window), int(sinks), int(trigger), int(aggregate), int(bool(check_stats)))
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -159,6 +166,8 @@ def _load() -> ctypes.CDLL:
                                            ctypes.POINTER(TriPhaseEvents), P]),
         "tri_status_string": (ctypes.c_char_p, [I]),
         "tri_selftest_bounded_wait": (I, [P, P, P]),
+        "tri_static_scratch_bytes": (S, []),
+        "tri_check_stats": (I, [P, P, P, I, I, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -318,6 +327,12 @@ def tri_compress_step(cache: KvCache, qbar, qabs, R, rope_base: float, deltas, b
     _check(code, "tri_compress_step")
 
 
+def tri_static_scratch_bytes() -> int:
+    """Bytes of the fixed device scratch built into the library (the
+    largest workspace tri_compress_step_static_scratch can serve)."""
+    return int(library().tri_static_scratch_bytes())
+
+
 def tri_compress_step_static_scratch(cache: KvCache, qbar, qabs, R, rope_base: float, deltas, budget: int,
                                      window: int, freed_ids, freed_count, idx_out=None, stream=None) -> None:
     """tri_compress_step without a workspace argument: the library's own
@@ -411,6 +426,22 @@ def tri_compress_step_distance(cache: KvCache, table, slot_pos, opt: TriStepOpti
         _ptr(idx_out, torch.int32, "idx_out", allow_none=True),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _events(events), _stream(stream))
     _check(code, "tri_compress_step_distance")
+
+
+def tri_check_stats(qbar, qabs, R, status, head_flags=None, stream=None) -> None:
+    """Check head statistics qbar f32 [L][Hq][D], qabs f32 [L][Hq][D/2],
+    R f32 [L][Hq]; per-head TRI_STATS_* bits go to head_flags (int32
+    [L][Hq], optional) and TRI_DEVFLAG_STATS to the status word on a failure."""
+    L, Hq, D = qbar.shape
+    if tuple(qabs.shape) != (L, Hq, D // 2) or tuple(R.shape) != (L, Hq):
+        raise ValueError("inconsistent statistics shapes")
+    if head_flags is not None and tuple(head_flags.shape) != (L, Hq):
+        raise ValueError("head_flags must be [L][Hq]")
+    code = library().tri_check_stats(
+        _ptr(qbar, torch.float32, "qbar"), _ptr(qabs, torch.float32, "qabs"), _ptr(R, torch.float32, "R"),
+        L, Hq, D, _ptr(head_flags, torch.int32, "head_flags", allow_none=True),
+        _ptr(status, torch.int32, "status"), _stream(stream))
+    _check(code, "tri_check_stats")
 
 
 def tri_sync_status(status, stream=None) -> int:

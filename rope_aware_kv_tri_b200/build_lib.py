@@ -20,7 +20,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libtriattn.so")
-SOURCES = ["tri_abi.cu", "calibrate.cu", "query.cu", "score.cu", "score_mma.cu", "evict.cu", "distance.cu", "tri_static_scratch.cu", "selftest.cu"]
+SOURCES = ["tri_abi.cu", "calibrate.cu", "query.cu", "score.cu", "score_mma.cu", "evict.cu", "distance.cu", "tri_static_scratch.cu", "selftest.cu", "stats_check.cu"]
 HEADERS = ["tri_device.cuh", "tri_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -868,6 +868,7 @@ __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictPara
     const int s = u / LH, rem = u % LH, l = rem / p.Hkv, h = rem % p.Hkv;
     const bool head0 = (l == 0 && h == 0);
     wait_prior_grid();
+    if (p.abort_word && __ldcg(p.abort_word) != 0) return;    // vetoed step: change nothing
     int len = p.lens[s];
     if (len < 0 || (int64_t)len > (int64_t)p.max_blocks * kBlockRows) {
         if (threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
@@ -1056,6 +1057,7 @@ __device__ void copy_out_rows(const MoveParams& p) {
 
 __global__ void __launch_bounds__(kMoveThreads, 3) move_kernel(const MoveParams p) {
     wait_prior_grid();
+    if (p.abort_word && __ldcg(p.abort_word) != 0) return;    // vetoed step: move nothing
     if (p.copy_out) {
         copy_out_rows(p);
         return;

@@ -25,7 +25,9 @@
 // copies them to the workspace, and writes the prefix offsets of the score
 // work items and of the freed-block list.  A sequence is compressed when its
 // length exceeds the trigger (at least the budget); when a device free list
-// is given it also reserves the list entries the freed ids will fill.
+// is given it also reserves the list entries the freed ids will fill.  When
+// the step's statistics check (stats_check.cu) vetoed the step, nothing is
+// planned: no work items, no freed blocks, no free-list entries.
 #include "tri_device.cuh"
 #include "tri_internal.h"
 
@@ -106,6 +108,8 @@ __device__ void plan_sequences(const QueryParams& p) {
     __shared__ int warp_tmp[kQueryThreads / 32];
     const int n_hg = p.Hkv / p.heads_per_tile;
     const int64_t max_len = (int64_t)p.max_blocks * kBlockRows;
+    // a step vetoed by the statistics check scores, selects and frees nothing
+    const bool vetoed = p.abort_word != nullptr && *p.abort_word != 0;
     int carry_items = 0, carry_freed = 0;
     for (int c0 = 0; c0 < p.S; c0 += kQueryThreads) {
         const int s = c0 + threadIdx.x;
@@ -119,7 +123,7 @@ __device__ void plan_sequences(const QueryParams& p) {
             p.len_ws[s] = len;
             const int nblk = (len + kBlockRows - 1) / kBlockRows;
             const bool compress = p.budget > 0;
-            const bool touched = !compress || len > p.trigger;
+            const bool touched = !vetoed && (!compress || len > p.trigger);
             const int scored = touched ? nblk : 0;
             items = p.L * n_hg * ((scored + kChunkBlocks - 1) / kChunkBlocks);
             if (compress && touched) nf = nblk - (p.budget + kBlockRows - 1) / kBlockRows;

@@ -52,7 +52,7 @@ WsLayout ws_layout(const tri_kv_desc* d, int budget, bool per_head = false) {
     w.idx = off;       off = align_up(off + U * (size_t)(budget > 0 ? budget : 0) * sizeof(int32_t));
     w.scratch_rows = scratch_rows_for(d, budget);
     const size_t per_unit = budget > 0 ? 1 : 0;
-    w.words = off;     off = align_up(off + 4 * sizeof(int32_t) * per_unit);   // scratch rows used, 0, free-list base
+    w.words = off;     off = align_up(off + 4 * sizeof(int32_t) * per_unit);   // scratch rows used, 0, free-list base, statistics veto
     w.info = off;      off = align_up(off + U * 4 * sizeof(int32_t) * per_unit);
     w.owner = off;     off = align_up(off + (size_t)w.scratch_rows * 2 * sizeof(int32_t));
     w.scratch = off;   off = align_up(off + (size_t)w.scratch_rows * 2 * kHeadDim * 2);
@@ -268,7 +268,7 @@ void set_step_plan(QueryParams& q, const tri_kv_desc* desc, uint8_t* ws, const W
 // the workspace (evict: select + plan + at-risk rows; copy-out; move).
 tri_status select_and_compact(const tri_kv_desc* desc, uint8_t* ws, const WsLayout& w, const tri_step_options& opt,
                               int trigger, const tri_free_list* free_list, int32_t* freed_ids, int32_t* idx_out,
-                              int32_t* slot_pos, bool pdl, cudaStream_t stream) {
+                              int32_t* slot_pos, bool pdl, cudaStream_t stream, const int32_t* veto = nullptr) {
     const int budget = opt.budget;
     EvictParams e = make_evict_params(desc);
     e.scores = reinterpret_cast<const float*>(ws + w.scores);
@@ -298,6 +298,7 @@ tri_status select_and_compact(const tri_kv_desc* desc, uint8_t* ws, const WsLayo
     e.scratch_rows = w.scratch_rows;
     // the evict kernel keeps two 512-thread CTAs per SM resident
     e.many_units = (int64_t)desc->S * desc->L * desc->Hkv > (int64_t)4 * device_sm_count() ? 1 : 0;
+    e.abort_word = veto;
     tri_status st;
     if ((st = cuda_status(launch_evict(e, stream, pdl))) != TRI_OK) return st;
     MoveParams mv = make_move_params(desc, reinterpret_cast<const int32_t*>(ws + w.idx), budget);
@@ -309,6 +310,7 @@ tri_status select_and_compact(const tri_kv_desc* desc, uint8_t* ws, const WsLayo
     mv.scratch_owner = reinterpret_cast<const int32_t*>(ws + w.owner);
     mv.scratch_used = reinterpret_cast<const int32_t*>(ws + w.words);
     mv.scratch_rows = w.scratch_rows;
+    mv.abort_word = veto;
     mv.copy_out = 1;
     if ((st = cuda_status(launch_move(mv, device_sm_count(), stream, pdl))) != TRI_OK) return st;
     mv.copy_out = 0;
@@ -429,7 +431,7 @@ tri_status tri_score_ex(const tri_kv_desc* desc, const float* qbar, const float*
 
 tri_status tri_select_topk(const tri_kv_desc* desc, const float* scores, int budget, int window, int32_t* idx,
                            int32_t* kept, cudaStream_t stream) {
-    const tri_step_options o = {budget, window, 0, 0, TRI_AGG_MEAN};
+    const tri_step_options o = {budget, window, 0, 0, TRI_AGG_MEAN, 0};
     return tri_select_topk_ex(desc, scores, &o, idx, kept, stream);
 }
 
@@ -496,7 +498,7 @@ tri_status tri_compress_step(tri_kv_desc* desc, const float* qbar, const float* 
                              int32_t* freed_ids, int32_t* freed_count, int32_t* idx_out, void* workspace,
                              size_t ws_bytes, const tri_phase_events* events, cudaStream_t stream) {
     if (!freed_ids || !freed_count) return TRI_ERR_INVALID;
-    const tri_step_options o = {budget, window, 0, 0, TRI_AGG_MEAN};
+    const tri_step_options o = {budget, window, 0, 0, TRI_AGG_MEAN, 0};
     return tri_compress_step_ex(desc, qbar, qabs, R, rope_base, deltas, n_deltas, &o, nullptr, freed_ids,
                                 freed_count, idx_out, workspace, ws_bytes, events, stream);
 }
@@ -528,10 +530,25 @@ tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const floa
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const WsLayout w = ws_layout(desc, budget, per_head);
     const int trigger = effective_trigger(*opt);
+    // The statistics check runs first and can veto the step (the word is
+    // read by the plan, the selection and the move kernels).
+    int32_t* veto = opt->check_stats ? reinterpret_cast<int32_t*>(ws + w.words) + 3 : nullptr;
+    if (veto) {
+        if ((st = cuda_status(cudaMemsetAsync(veto, 0, sizeof(int32_t), stream))) != TRI_OK) return st;
+        StatsCheckParams c{};
+        c.qbar = qbar;
+        c.qabs = qabs;
+        c.R = R;
+        c.n_heads = (int64_t)desc->L * desc->Hkv * desc->G;
+        c.status = desc->status;
+        c.abort_word = veto;
+        if ((st = cuda_status(launch_check_stats(c, stream))) != TRI_OK) return st;
+    }
     QueryParams q = make_query_params(desc, qbar, qabs, R, rope_base, deltas, n_deltas,
                                       reinterpret_cast<float*>(ws + w.qeff), reinterpret_cast<float*>(ws + w.wts));
     q.per_head = per_head ? 1 : 0;
     set_step_plan(q, desc, ws, w, budget, trigger, freed_count, free_list);
+    q.abort_word = veto;
     if ((st = cuda_status(launch_query(q, stream))) != TRI_OK) return st;
     if (events) record(events->after_query, stream);
 
@@ -545,11 +562,28 @@ tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const floa
         return st;
     if (events) record(events->after_score, stream);
 
-    if ((st = select_and_compact(desc, ws, w, *opt, trigger, free_list, freed_ids, idx_out, nullptr, pdl, stream)) !=
-        TRI_OK)
+    if ((st = select_and_compact(desc, ws, w, *opt, trigger, free_list, freed_ids, idx_out, nullptr, pdl, stream,
+                                 veto)) != TRI_OK)
         return st;
     if (events) record(events->after_evict, stream);
     return TRI_OK;
+}
+
+tri_status tri_check_stats(const float* qbar, const float* qabs, const float* R, int L, int Hq, int D,
+                           int32_t* head_flags, int32_t* status, cudaStream_t stream) {
+    if (L < 1 || Hq < 1 || (int64_t)L * Hq > INT_MAX) return TRI_ERR_INVALID;
+    if (D != TRI_HEAD_DIM) return TRI_ERR_UNSUPPORTED;
+    if (check_stats(qbar, qabs, R) != TRI_OK || !status || !aligned(status, 4) ||
+        (head_flags && !aligned(head_flags, 4)))
+        return TRI_ERR_INVALID;
+    StatsCheckParams c{};
+    c.qbar = qbar;
+    c.qabs = qabs;
+    c.R = R;
+    c.n_heads = (int64_t)L * Hq;
+    c.head_flags = head_flags;
+    c.status = status;
+    return cuda_status(launch_check_stats(c, stream));
 }
 
 tri_status tri_distance_table(int L, int Hkv, int G, int D, const float* qbar, const float* kbar, double rope_base,
@@ -669,6 +703,7 @@ tri_status tri_sync_status(int32_t* status, cudaStream_t stream) {
     if (h & TRI_DEVFLAG_BOUNDS) return TRI_ERR_DEVICE_BOUNDS;
     if (h & TRI_DEVFLAG_TIMEOUT) return TRI_ERR_TIMEOUT;
     if (h & TRI_DEVFLAG_FREELIST) return TRI_ERR_FREELIST;
+    if (h & TRI_DEVFLAG_STATS) return TRI_ERR_STATS;
     if (h & TRI_DEVFLAG_NONFINITE) return TRI_ERR_NONFINITE;
     return TRI_OK;
 }
@@ -684,6 +719,7 @@ const char* tri_status_string(tri_status s) {
         case TRI_ERR_NONFINITE: return "NaN score";
         case TRI_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
         case TRI_ERR_FREELIST: return "device free list had too few entries or too little room";
+        case TRI_ERR_STATS: return "head statistics failed the sanity check";
         default: return "unknown status";
     }
 }

@@ -66,6 +66,7 @@ struct QueryParams {
     int32_t* fl_count;        // free list to push the freed ids on, or null
     int fl_capacity;
     int32_t* fl_base;         // [1] out: first list entry of this step's ids, -1 if no room
+    const int32_t* abort_word; // non-zero: the statistics check vetoed the step (plan nothing), or null
     int32_t* status;
 };
 cudaError_t launch_query(const QueryParams& p, cudaStream_t stream);
@@ -137,6 +138,7 @@ struct EvictParams {
     int32_t* scratch_owner;    // [2][scratch_rows]: unit and source row of each scratch row
     int scratch_rows;          // capacity of the scratch in rows
     int many_units;            // several waves of unit CTAs: long at-risk prefixes compact in place
+    const int32_t* abort_word; // non-zero: the step was vetoed, touch nothing; or null
 };
 cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream, bool pdl = false);
 
@@ -158,6 +160,7 @@ struct MoveParams {
     const int32_t* scratch_used;   // [1] scratch rows handed out
     int scratch_rows;
     int copy_out;              // 1: copy at-risk sources to the scratch; 0: move rows
+    const int32_t* abort_word; // non-zero: the step was vetoed, move nothing; or null
 };
 cudaError_t launch_move(const MoveParams& p, int num_sms, cudaStream_t stream, bool pdl = false);
 
@@ -216,6 +219,18 @@ struct ReserveParams {
     int32_t* status;
 };
 cudaError_t launch_reserve(const ReserveParams& p, cudaStream_t stream);
+
+// ---------------------------------------------------------- stats check
+struct StatsCheckParams {
+    const float* qbar;        // [n_heads][D]
+    const float* qabs;        // [n_heads][D/2]
+    const float* R;           // [n_heads]
+    int64_t n_heads;
+    int32_t* head_flags;      // [n_heads] TRI_STATS_* bits, or null
+    int32_t* status;          // TRI_DEVFLAG_STATS raised here on a failure
+    int32_t* abort_word;      // set to non-zero on a failure (a step's veto), or null
+};
+cudaError_t launch_check_stats(const StatsCheckParams& p, cudaStream_t stream);
 
 // ------------------------------------------------------------- calibrate
 cudaError_t launch_calibrate(const float* q, int N, int L, int Hq, float* qbar, float* qabs, float* R,

@@ -37,6 +37,12 @@ def test_exports_every_declared_function(lib):
         assert hasattr(lib, n), n
 
 
+def test_static_scratch_size_matches_header(lib):
+    m = re.search(r"#define\s+TRI_STATIC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", open(HEADER).read())
+    assert m, "TRI_STATIC_SCRATCH_BYTES not found in the header"
+    assert tri.tri_static_scratch_bytes() == int(m.group(1)) << int(m.group(2))
+
+
 def test_status_strings(lib):
     assert tri.tri_status_string(0) == "ok"
     for code in range(1, 9):
@@ -261,3 +267,21 @@ def test_distance_alignment_rules(lib):
     d = _desc()
     assert lib.tri_score_distance(ctypes.byref(d), FAKE, 100, FAKE + 4, FAKE, None) == tri.TRI_ERR_INVALID
     assert lib.tri_score_distance(ctypes.byref(d), FAKE, 100, FAKE, FAKE + 8, None) == tri.TRI_ERR_INVALID
+
+
+def test_check_stats_rejects(lib):
+    assert lib.tri_check_stats(None, FAKE, FAKE, 2, 4, 128, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_check_stats(FAKE, FAKE, FAKE, 0, 4, 128, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_check_stats(FAKE, FAKE, FAKE, 2, 0, 128, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_check_stats(FAKE, FAKE, FAKE, 2, 4, 64, None, FAKE, None) == tri.TRI_ERR_UNSUPPORTED
+    assert lib.tri_check_stats(FAKE, FAKE, FAKE, 2, 4, 128, None, None, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_check_stats(FAKE, FAKE, FAKE, 2, 4, 128, FAKE + 2, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_check_stats(FAKE + 1, FAKE, FAKE, 2, 4, 128, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert lib.tri_check_stats(FAKE, FAKE, FAKE, 1 << 16, 1 << 16, 128, None, FAKE, None) == tri.TRI_ERR_INVALID
+    assert tri.tri_status_string(tri.TRI_ERR_STATS) == "head statistics failed the sanity check"
+
+
+def test_step_options_mirror_has_check_stats(lib):
+    o = tri.step_options(64, 8, check_stats=True)
+    assert o.check_stats == 1 and ctypes.sizeof(o) == 6 * ctypes.sizeof(ctypes.c_int)
+    assert tri.step_options(64, 8).check_stats == 0
