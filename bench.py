@@ -14,6 +14,9 @@ whole step against the measured B200 copy bandwidth.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
     torchrun --nproc-per-node N bench.py --gpus N ...   (one rank per GPU)
 
+--gpus N > 1 without torchrun starts the N ranks itself (one process per
+GPU, NCCL); under torchrun WORLD_SIZE must equal --gpus.
+
 Timing: each timed step restores the kept region of the cache and flushes L2
 (256 MiB write) outside CUDA events that bracket only the tri_compress_step
 launches; the K/V pools (4.3 GB) are larger than L2 as well.  The timed loop
@@ -45,7 +48,7 @@ L2_FLUSH_BYTES = 256 << 20
 SCORE_SOURCES = ["score.cu", "tri_device.cuh", "tri_internal.h"]
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
@@ -71,7 +74,7 @@ def parse_args():
                     help="decode loop: time each round's phases with library events (serialises launches)")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling cases of the same kernels)")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 # ----------------------------------------------------------------- helpers
@@ -179,20 +182,94 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def dist_setup(args):
+def dist_setup(args, backend="nccl"):
+    """Rank, world and process group of this process.  Under torchrun (or a
+    rank spawned by ``spawn_ranks``) the world comes from WORLD_SIZE, which
+    must equal --gpus; a single process has world 1.  ``backend`` "nccl"
+    binds the process to GPU LOCAL_RANK; "gloo" (host-only tests) does not."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if "WORLD_SIZE" in os.environ and world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU")
     if world > 1:
         import torch.distributed as dist
         if args.impl == "reference":
             return world, rank, local, None
-        import torch
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            import torch
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         return world, rank, local, dist
     return world, rank, local, None
+
+
+def rank_plan(args, world, rank):
+    """The workload one rank runs: (config, seed, heads_mode).
+
+    --shard sequences (default): every rank runs its own independent cache
+    of the full workload shape, seeded per rank (weak scaling).  --shard
+    heads: the KV heads of one cache are split over the ranks (each keeps
+    its slice of heads, and their query heads, for every sequence), every
+    rank seeded apart (strong scaling)."""
+    from workload import CONFIGS
+    from rope_aware_kv_tri_b200.sharding import shard_heads, shard_seed
+    cfg = CONFIGS[args.workload]
+    if args.layers > 0:
+        cfg = cfg.replace(L=args.layers, name=f"{cfg.name} (L={args.layers})")
+    heads_mode = args.shard == "heads" and world > 1
+    if heads_mode:
+        cfg = cfg.replace(Hkv=len(shard_heads(cfg.Hkv, world, rank)))
+    seed = shard_seed(cfg.seed, rank) if world > 1 else cfg.seed
+    return cfg, seed, heads_mode
+
+
+def job_summary(dist, step_ms_total, keys_per_step, freed_per_step, steps, heads_mode, device=None):
+    """Reduce one rank's timed steps to the job's figures: the slowest
+    rank's time, all ranks' keys and freed blocks, and (head sharding)
+    whether every rank freed the same number of blocks.  Every rank takes
+    the same collective steps in the same order."""
+    from rope_aware_kv_tri_b200.sharding import freed_consistent, keys_per_second, reduce_job
+    total_ms, job_keys, job_freed = reduce_job(dist, step_ms_total, keys_per_step, freed_per_step, device)
+    freed_same = freed_consistent(dist, freed_per_step, device) if heads_mode else None
+    world = dist.get_world_size() if dist is not None else 1
+    return {"value": keys_per_second(job_keys, steps, total_ms), "ms_per_step": total_ms / steps,
+            "job_keys": job_keys, "job_freed": job_freed, "freed_same": freed_same, "n_gpus": world,
+            "scaling": "strong" if heads_mode else "weak"}
+
+
+def _free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def _spawned_rank(rank, world, port, argv, runner, backend):
+    os.environ.update({"RANK": str(rank), "LOCAL_RANK": str(rank), "WORLD_SIZE": str(world),
+                       "LOCAL_WORLD_SIZE": str(world), "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+    main(argv, runner=runner, backend=backend)
+
+
+def spawn_ranks(args, argv, runner=None, backend="nccl"):
+    """--gpus N > 1 without torchrun: start N ranks on this node, one process
+    per GPU (rank r on GPU r), with the same arguments; rank 0 prints the
+    job's line.  Returns the worst exit code."""
+    import torch.multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    port = _free_port()
+    procs = [ctx.Process(target=_spawned_rank, args=(r, args.gpus, port, argv, runner, backend))
+             for r in range(args.gpus)]
+    for p in procs:
+        p.start()
+    codes = []
+    for p in procs:
+        p.join()
+        codes.append(p.exitcode if p.exitcode is not None else 1)
+    return max(codes, key=abs)
 
 
 def unit_rows(pool, table_row, length, l, h):
@@ -290,17 +367,10 @@ def run_ours(args, world, rank, local, dist):
     build_lib.build()
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    cfg = CONFIGS[args.workload]
-    if args.layers > 0:
-        cfg = cfg.replace(L=args.layers, name=f"{cfg.name} (L={args.layers})")
     if args.workload == "decode16":
-        return run_decode(args, world, rank, local, dist, cfg)
-    from rope_aware_kv_tri_b200.sharding import freed_consistent, keys_per_second, reduce_job, shard_heads, shard_seed
-    heads_mode = args.shard == "heads" and world > 1
-    if heads_mode:
-        # this rank's slice of the KV heads (and their query heads) of every sequence
-        cfg = cfg.replace(Hkv=len(shard_heads(cfg.Hkv, world, rank)))
-    wl = make_workload(cfg, device=dev, seed=shard_seed(cfg.seed, rank) if world > 1 else cfg.seed)
+        return run_decode(args, world, rank, local, dist, rank_plan(args, world, rank)[0])
+    cfg, seed, heads_mode = rank_plan(args, world, rank)
+    wl = make_workload(cfg, device=dev, seed=seed)
     L, Hkv, G, Hq, S = cfg.L, cfg.Hkv, cfg.G, cfg.Hq, cfg.S
     B, W = cfg.budget, cfg.window
     stream = torch.cuda.current_stream(dev)
@@ -442,10 +512,9 @@ def run_ours(args, world, rank, local, dist):
     query_ms = [e[0].elapsed_time(e[1]) for e in pevs]
     score_ms = [e[1].elapsed_time(e[2]) for e in pevs]
     evict_ms = [e[2].elapsed_time(e[3]) for e in pevs]
-    total_ms, job_keys, job_freed = reduce_job(dist, sum(step_ms), keys_per_step, freed_per_step, dev)
-    freed_same = freed_consistent(dist, freed_per_step, dev) if heads_mode else None
-    value = keys_per_second(job_keys, args.steps, total_ms)
-    ms_per_step = total_ms / args.steps
+    job = job_summary(dist, sum(step_ms), keys_per_step, freed_per_step, args.steps, heads_mode, dev)
+    value, ms_per_step = job["value"], job["ms_per_step"]
+    job_freed, freed_same = job["job_freed"], job["freed_same"]
 
     peak, peak_kind = measured_peak()
     bytes_per_key = 12 if distance else 256     # distance: position + table entry + score; keys: the bf16 key
@@ -486,9 +555,9 @@ def run_ours(args, world, rank, local, dist):
 
     clk = clocks.summary()
     out = {
-        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": job["n_gpus"], "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
-        "scaling": "strong" if heads_mode else "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "scaling": job["scaling"], "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "seq_lens": lens,
                    "budget": B, "window": W, "rope_base": cfg.base, "deltas": wl.deltas,
                    "sinks": args.sinks, "trigger": trig, "aggregate": args.aggregate,
@@ -536,6 +605,11 @@ def run_decode(args, world, rank, local, dist, cfg):
     fl = tri.FreeList.from_ids(wl.free_blocks, wl.num_blocks, dev)
     n_new = torch.full((S,), cfg.decode_append, dtype=torch.int32, device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    # kept slots of every unit (an optional output of the step), to count the
+    # rows each round moves once the round is over
+    idx = torch.empty(S, L, Hkv, B, dtype=torch.int32, device=dev)
+    ident = torch.arange(B, dtype=torch.int32, device=dev)
+    peak, peak_kind = measured_peak()
     rounds, total_ms, total_keys = [], 0.0, 0
     clocks = ClockSampler(local)
     clocks.start()
@@ -553,17 +627,23 @@ def run_decode(args, world, rank, local, dist, cfg):
         pev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if args.phases else None
         torch.cuda.synchronize(dev)
         a.record()
-        tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, free_list=fl, events=pev)
+        tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, free_list=fl, idx_out=idx,
+                                 events=pev)
         b.record()
         torch.cuda.synchronize(dev)
         if tri.tri_sync_status(cache.status) != tri.TRI_OK:
             raise RuntimeError(f"device status flag raised in decode round {r}")
         ms = a.elapsed_time(b)
         trig = max(args.trigger, B)
-        keys = sum(n for n in lens if n > trig) * L * Hkv
+        compressed = [s for s in range(S) if lens[s] > trig]
+        keys = sum(lens[s] for s in compressed) * L * Hkv
+        moved = int((idx[compressed] != ident).sum().item()) if compressed else 0
+        step_bytes = keys * 256 + moved * 4 * 256
         freed = int(fl.count.item()) - free_before
         rounds.append({"round": r, "keys": keys, "ms": round(ms, 4), "keys_per_s": round(keys / (ms / 1e3), 1),
-                       "k_read_gbs": round(keys * 256 / (ms / 1e3) / 1e9, 1), "freed_blocks": freed,
+                       "k_read_gbs": round(keys * 256 / (ms / 1e3) / 1e9, 1), "moved_rows": moved,
+                       "step_bytes": step_bytes, "step_gbs": round(step_bytes / (ms / 1e3) / 1e9, 1),
+                       "frac": round(step_bytes / (ms / 1e3) / 1e9 / peak, 4), "freed_blocks": freed,
                        "mean_len_before": round(sum(lens) / S, 1)})
         if pev is not None:
             rounds[-1]["phase_ms"] = {"query": round(pev[0].elapsed_time(pev[1]), 4),
@@ -574,7 +654,10 @@ def run_decode(args, world, rank, local, dist, cfg):
     clocks.stop()
     t_job, k_job, _ = reduce_job(dist, total_ms, total_keys, 0, dev)
     value = keys_per_second(k_job, 1, t_job)
-    peak, peak_kind = measured_peak()
+    steady = rounds[1:] if len(rounds) > 1 else rounds
+    steady_ms = sum(x["ms"] for x in steady)
+    steady_bytes = sum(x["step_bytes"] for x in steady)
+    all_bytes = sum(x["step_bytes"] for x in rounds)
     out = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": cfg.decode_rounds,
         "warmup": 0, "ms_per_step": round(t_job / cfg.decode_rounds, 5), "higher_is_better": True,
@@ -584,7 +667,18 @@ def run_decode(args, world, rank, local, dist, cfg):
                    "free_list": "device (tri_reserve_blocks pops, the step pushes; no host read of freed ids)",
                    "timing": "CUDA events around each round's tri_compress_step_ex; appends untimed",
                    "rounds": rounds},
-        "roofline": {"bound": "hbm", "peak": peak, "unit": "GB/s", "peak_source": peak_kind,
+        "roofline": {"bound": "hbm", "achieved": round(all_bytes / (total_ms / 1e3) / 1e9, 1), "peak": peak,
+                     "unit": "GB/s", "frac": round(all_bytes / (total_ms / 1e3) / 1e9 / peak, 4),
+                     "traffic": None, "kernel": "whole step (score + select + compaction)",
+                     "bytes": "per round: cached keys x 256 B read + moved rows x 1024 B (K and V read and "
+                              "written), summed over the rounds",
+                     "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                     else "fallback 6650 GB/s",
+                     "steady_rounds": {"rounds": len(steady), "ms_mean": round(steady_ms / max(len(steady), 1), 4),
+                                       "moved_rows_mean": round(sum(x["moved_rows"] for x in steady)
+                                                                / max(len(steady), 1), 1),
+                                       "achieved": round(steady_bytes / (steady_ms / 1e3) / 1e9, 1),
+                                       "frac": round(steady_bytes / (steady_ms / 1e3) / 1e9 / peak, 4)},
                      "achieved_k_read_first_round": rounds[0]["k_read_gbs"] if rounds else None},
         "gpu_launches": 5 * cfg.decode_rounds, "clocks": clocks.summary(),
     }
@@ -835,14 +929,21 @@ def run_reference(args, world, rank):
     print(json.dumps(out), flush=True)
 
 
-def main():
-    args = parse_args()
-    world, rank, local, dist = dist_setup(args)
+def main(argv=None, runner=None, backend="nccl"):
+    """``runner(args, world, rank, local, dist)`` runs one rank's measurement
+    (default: run_ours)."""
+    args = parse_args(argv)
+    if args.impl != "reference" and args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        code = spawn_ranks(args, argv if argv is not None else sys.argv[1:], runner, backend)
+        if code:
+            raise SystemExit(code)
+        return
+    world, rank, local, dist = dist_setup(args, backend)
     if args.impl == "reference":
         run_reference(args, world, rank)
         return
     try:
-        run_ours(args, world, rank, local, dist)
+        (runner or run_ours)(args, world, rank, local, dist)
     finally:
         if dist is not None:
             dist.destroy_process_group()

@@ -11,6 +11,7 @@ import ctypes
 import os
 import shutil
 import subprocess
+import threading
 from typing import Sequence, Tuple
 
 import numpy as np
@@ -20,25 +21,31 @@ SRC = os.path.join(HERE, "tri_oracle_c.c")
 LIB = os.path.join(HERE, "_lib", "libtrioracle.so")
 
 _lib = None
+_lock = threading.RLock()
 
 
 def build(force: bool = False) -> str:
-    """Compile the C oracle (plain -O2, no fast-math) if missing or stale."""
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+    """Compile the C oracle (plain -O2, no fast-math) if missing or stale.
+    Safe to call from several threads or processes at once: each compiles
+    to its own temporary file and renames it into place."""
+    with _lock:
+        if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= os.path.getmtime(SRC):
+            return LIB
+        cc = shutil.which("gcc") or shutil.which("cc")
+        if cc is None:
+            raise RuntimeError("no C compiler for the C oracle")
+        os.makedirs(os.path.dirname(LIB), exist_ok=True)
+        tmp = f"{LIB}.{os.getpid()}.tmp"
+        subprocess.run([cc, "-O2", "-fPIC", "-shared", "-o", tmp, SRC, "-lm"], check=True, capture_output=True)
+        os.replace(tmp, LIB)
         return LIB
-    cc = shutil.which("gcc") or shutil.which("cc")
-    if cc is None:
-        raise RuntimeError("no C compiler for the C oracle")
-    os.makedirs(os.path.dirname(LIB), exist_ok=True)
-    tmp = LIB + ".tmp"
-    subprocess.run([cc, "-O2", "-fPIC", "-shared", "-o", tmp, SRC, "-lm"], check=True, capture_output=True)
-    os.replace(tmp, LIB)
-    return LIB
 
 
 def _load():
     global _lib
-    if _lib is None:
+    with _lock:
+        if _lib is not None:
+            return _lib
         lib = ctypes.CDLL(build())
         P, I = ctypes.c_void_p, ctypes.c_int
         lib.tri_oracle_unit.restype = I

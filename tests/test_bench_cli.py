@@ -37,7 +37,7 @@ def test_reference_arm_prints_the_contract_line():
 
 
 def test_reference_arm_other_ranks_exit_quietly():
-    r = _run(["--impl", "reference", "--workload", "head1_t4096", "--steps", "1", "--warmup", "0"],
+    r = _run(["--impl", "reference", "--workload", "head1_t4096", "--steps", "1", "--warmup", "0", "--gpus", "2"],
              env_extra={"RANK": "1", "LOCAL_RANK": "1", "WORLD_SIZE": "2"})
     assert r.returncode == 0, r.stderr[-2000:]
     assert r.stdout.strip() == ""
@@ -102,3 +102,61 @@ def test_reference_arm_times_the_requested_variant():
             assert d["config"]["aggregate"] == "max" and d["config"]["sinks"] == 2
         else:
             assert d["config"]["score_mode"] == "distance"
+
+
+def _stub_runner(args, world, rank, local, dist):
+    """One rank of ``bench.main`` with the GPU step replaced by a stand-in
+    timing (rank r takes 10 + r ms over the timed steps) and a freed count
+    derived from the rank's own plan; everything else is bench.py's own
+    per-rank plan and job reduction over the process group."""
+    import bench
+    cfg, seed, heads_mode = bench.rank_plan(args, world, rank)
+    keys_per_step = sum(cfg.lens) * cfg.L * cfg.Hkv
+    freed_per_step = sum(-(-n // 16) - -(-min(n, cfg.budget) // 16) for n in cfg.lens)
+    job = bench.job_summary(dist, 10.0 + rank, keys_per_step, freed_per_step, args.steps, heads_mode)
+    plans = [None] * world
+    dist.all_gather_object(plans, (cfg.Hkv, seed))
+    if rank == 0:
+        print(json.dumps({"n_gpus": job["n_gpus"], "scaling": job["scaling"], "value": job["value"],
+                          "ms_per_step": job["ms_per_step"], "job_keys": job["job_keys"],
+                          "job_freed": job["job_freed"], "freed_same": job["freed_same"], "plans": plans}),
+              flush=True)
+
+
+def _spawned_bench(argv):
+    code = ("import sys, json\n"
+            f"sys.path.insert(0, {ROOT!r})\n"
+            "import bench\n"
+            "from tests.test_bench_cli import _stub_runner\n"
+            f"bench.main({argv!r}, runner=_stub_runner, backend='gloo')\n")
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    return subprocess.run([sys.executable, "-c", code], cwd=ROOT, env=env, capture_output=True, text=True,
+                          timeout=300)
+
+
+def test_gpus_flag_spawns_that_many_ranks_with_head_sharding():
+    r = _spawned_bench(["--gpus", "2", "--shard", "heads", "--steps", "4"])
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout                # rank 0 alone prints
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["scaling"] == "strong"
+    # the 32x8-head workload's KV heads split 4 + 4, each rank seeded apart
+    assert [p[0] for p in d["plans"]] == [4, 4] and d["plans"][0][1] != d["plans"][1][1]
+    assert d["ms_per_step"] == 11.0 / 4                      # the slowest rank's time
+    assert d["job_keys"] == 2 * 32768 * 32 * 4              # both ranks' keys
+    assert d["freed_same"] is True and d["job_freed"] == 2 * 1920
+    assert d["value"] == d["job_keys"] * 4 / 0.011
+
+
+def test_gpus_flag_with_sequence_sharding_is_weak_scaling():
+    r = _spawned_bench(["--gpus", "2", "--steps", "2"])
+    assert r.returncode == 0, r.stderr[-3000:]
+    d = json.loads([ln for ln in r.stdout.splitlines() if ln.startswith("{")][0])
+    assert d["n_gpus"] == 2 and d["scaling"] == "weak" and d["freed_same"] is None
+    assert [p[0] for p in d["plans"]] == [8, 8] and d["job_keys"] == 2 * 32768 * 32 * 8
+
+
+def test_world_size_must_match_gpus_flag():
+    r = _run(["--gpus", "4", "--steps", "1"], env_extra={"WORLD_SIZE": "2", "RANK": "0", "LOCAL_RANK": "0"})
+    assert r.returncode != 0 and "WORLD_SIZE=2" in (r.stderr + r.stdout)
