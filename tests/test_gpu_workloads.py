@@ -37,6 +37,25 @@ def _built():
 def test_decode_loop_two_worlds():
     cfg = CONFIGS["decode16"].replace(L=2, Hkv=4, G=2, lens=[0] * 4, lens_range=(300, 700), budget=256, window=32,
                                   decode_append=64, decode_rounds=4, n_samples=256)
+    _two_worlds(cfg)
+
+
+def test_decode_loop_many_units_in_place_prefixes():
+    """The decode loop's steady rounds at a launch of several waves of unit
+    CTAs ([GeoTrick] "Solving the Memory Fragmentation Problem": compaction
+    every ~128 decode steps).  Caches sit at B + 128 slots when compressed,
+    so the 128 evicted slots fall among ~2000 kept rows that all move; with
+    more units than four per SM, prefixes longer than the scratch rule allows
+    are packed in place by their selection CTA.  Compared with the oracle's
+    world row for row after every round."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cfg = CONFIGS["decode16"].replace(L=16, Hkv=4, G=2, lens=[0] * 10, lens_range=(2048, 2048), budget=2048,
+                                  window=128, decode_append=128, decode_rounds=2, n_samples=256)
+    assert cfg.S * cfg.L * cfg.Hkv > 4 * sms            # several waves of selection CTAs
+    _two_worlds(cfg)
+
+
+def _two_worlds(cfg):
     cpu = make_workload(cfg, device="cpu")
     G, budget, window = cfg.G, cfg.budget, cfg.window
     # GPU world: same starting state
@@ -99,8 +118,27 @@ def test_decode_loop_two_worlds():
         gtable.copy_(cpu.block_table.to(DEV))
 
 
-def _full_size(name, sample_units, check_all_rows):
+def _step_ex(wl, stats, budget, window, aggregate):
+    """One tri_compress_step_ex with the given aggregation on the workload's
+    own tensors (modified in place)."""
+    cache = cache_of(wl)
+    S, L, Hkv = wl.cfg.S, wl.cfg.L, wl.cfg.Hkv
+    opt = tri.step_options(budget, window, aggregate=aggregate)
+    ws = tri.alloc_workspace(cache, opt)
+    freed = torch.full((S * wl.max_blocks,), -7, dtype=torch.int32, device=DEV)
+    count = torch.full((1,), -7, dtype=torch.int32, device=DEV)
+    idx = torch.full((S, L, Hkv, budget), -7, dtype=torch.int32, device=DEV)
+    tri.tri_compress_step_ex(cache, *stats, wl.cfg.base, wl.deltas, opt, ws, freed_ids=freed, freed_count=count,
+                             idx_out=idx)
+    code = tri.tri_sync_status(cache.status)
+    n = int(count.item())
+    return {"status": code, "freed": freed[:n].cpu().tolist(), "idx": idx}
+
+
+def _full_size(name, sample_units, check_all_rows, aggregate="mean", layers=None):
     cfg = CONFIGS[name]
+    if layers is not None:
+        cfg = cfg.replace(L=layers)
     wl = make_workload(cfg, device=DEV, seed=0)
     stats = gpu_stats(wl)
     budget, window = cfg.budget, cfg.window
@@ -120,12 +158,13 @@ def _full_size(name, sample_units, check_all_rows):
     # scores of the sampled units from tri_score on the untouched cache
     cache0 = cache_of(wl, seq_len=wl.seq_len.clone())
     max_len = wl.max_blocks * 16
-    ws0 = tri.alloc_workspace(cache0, 1)
+    agg = tri.TRI_AGG_MAX if aggregate == "max" else tri.TRI_AGG_MEAN
+    ws0 = tri.alloc_workspace(cache0, tri.step_options(1, 0, aggregate=agg))
     scores = torch.empty(S, L, Hkv, max_len, device=DEV)
-    tri.tri_score(cache0, *stats, cfg.base, wl.deltas, scores, ws0)
+    tri.tri_score_ex(cache0, *stats, cfg.base, wl.deltas, agg, scores, ws0)
     assert tri.tri_sync_status(cache0.status) == tri.TRI_OK
     del ws0
-    out = run_step(wl, stats, budget, window)
+    out = run_step(wl, stats, budget, window) if aggregate == "mean" else _step_ex(wl, stats, budget, window, agg)
     assert out["status"] == tri.TRI_OK
     assert wl.seq_len.cpu().tolist() == kept
     assert out["freed"] == freed_expected(wl.block_table, lens, kept)
@@ -153,7 +192,7 @@ def _full_size(name, sample_units, check_all_rows):
                            vals0[u][ui].view(torch.int16))
         ref_stats = oracle_stats(wl, l, slice(h * G, (h + 1) * G))
         ref = oracle.unit_scores(keys0[u].double().cpu().numpy(), *ref_stats, int(wl.cur_pos[s]), wl.deltas,
-                                 cfg.base)
+                                 cfg.base, aggregate=aggregate)
         err = check_scores(scores[s, l, h, :n].cpu().numpy(), ref)
         differ = check_selection(ui.cpu().numpy(), ref, n, budget, window)
         print(f"{name} unit {u}: worst score error/floor {err:.2e}, {differ} slots differ in the cut band")
@@ -169,3 +208,17 @@ def test_full_size_long_context_T131072_B4096():
 
 def test_full_size_wide_64L_G8_4x65536():
     _full_size("l64h8g8_4x64k", sample_units=4, check_all_rows=False)
+
+
+def test_full_size_max_over_group_32L_8H_T32768_B2048():
+    """The benchmark's headline shape with the maximum over the GQA group:
+    G = 4 runs on the tensor-core kernel, every (layer, block) stage of the
+    persistent CTAs' ring and every accumulator and coefficient switch of a
+    whole launch; all rows bit-exact, sampled units score by score."""
+    _full_size("l32h8_t32k", sample_units=6, check_all_rows=True, aggregate="max")
+
+
+def test_full_size_max_over_group_G8_4x65536():
+    """G = 8 (the widest group) on the tensor-core kernel: 16 layers of the
+    64-layer, 4 x 65536 workload."""
+    _full_size("l64h8g8_4x64k", sample_units=4, check_all_rows=True, aggregate="max", layers=16)
