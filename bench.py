@@ -45,7 +45,6 @@ UNIT = "keys/s"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 7700.0
 L2_FLUSH_BYTES = 256 << 20
-SCORE_SOURCES = ["score.cu", "tri_device.cuh", "tri_internal.h"]
 
 
 def parse_args(argv=None):
@@ -89,18 +88,29 @@ def measured_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def score_source_hash() -> str:
+# Sources of each kernel whose DRAM traffic record is kept under profiles/.
+KERNEL_SOURCES = {
+    "score_kernel": ["score.cu", "score_device.cuh", "tri_device.cuh", "tri_internal.h"],
+    "select_compact_kernel": ["select_compact.cu", "select_device.cuh", "tri_device.cuh", "tri_internal.h"],
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for name in SCORE_SOURCES:
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(ROOT, "rope_aware_kv_tri_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic_per_key():
-    """DRAM bytes per scored key of the score kernel from the committed ncu
-    summary, if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "score_kernel_traffic.txt")
+def recorded_traffic_per_launch(kernel: str, keys: int, moved_rows: int):
+    """DRAM bytes of one launch of ``kernel`` on this workload, from the
+    committed ncu record (bytes per scored key and per moved row, taken on a
+    smaller case of the same kernel), if that record was taken on the
+    kernel's current source; else None."""
+    if kernel not in KERNEL_SOURCES:
+        return None
+    path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.txt")
     try:
         kv = {}
         with open(path) as f:
@@ -108,9 +118,9 @@ def recorded_traffic_per_key():
                 if "=" in line and not line.lstrip().startswith("#"):
                     k, v = line.split("=", 1)
                     kv[k.strip()] = v.strip()
-        if kv.get("source_sha256") != score_source_hash():
+        if kv.get("source_sha256") != kernel_source_hash(kernel):
             return None
-        return float(kv["dram_bytes_per_key"])
+        return round(float(kv["dram_bytes_per_key"]) * keys + float(kv.get("dram_bytes_per_moved_row", 0)) * moved_rows)
     except Exception:
         return None
 
@@ -395,6 +405,7 @@ def run_ours(args, world, rank, local, dist):
     distance = args.score_mode == "distance"
     opt = tri.step_options(B, W, args.sinks, args.trigger,
                            tri.TRI_AGG_MAX if args.aggregate == "max" else tri.TRI_AGG_MEAN)
+    fused = tri.tri_step_is_fused(cache, opt)
     ws = tri.alloc_workspace(cache, opt)
     freed = torch.empty(S * wl.max_blocks, dtype=torch.int32, device=dev)
     count = torch.empty(1, dtype=torch.int32, device=dev)
@@ -521,23 +532,29 @@ def run_ours(args, world, rank, local, dist):
     k_bytes = keys_per_step * bytes_per_key
     moved_bytes = moved * 4 * 256
     score_mean = statistics.mean(score_ms)
-    achieved = k_bytes / (score_mean / 1e3) / 1e9
-    tpk = recorded_traffic_per_key()
+    kernel = "distance_score_kernel" if distance else ("score_mma_kernel" if args.aggregate == "max"
+                                                       else "score_kernel")
+    kernel_bytes = k_bytes
+    what = "the score kernel"
+    achieved = kernel_bytes / (score_mean / 1e3) / 1e9
+    tpl = recorded_traffic_per_launch(kernel, keys_per_step, moved) if not variant and not distance else None
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                "frac": round(achieved / peak, 4),
-                "traffic": (round(tpk * keys_per_step) if tpk and not variant and not distance else None),
-                "kernel": "distance_score_kernel" if distance else "score_kernel", "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+                "frac": round(achieved / peak, 4), "traffic": tpl, "kernel": kernel,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s",
-                "algorithmic_bytes_per_launch": k_bytes, "ms_per_launch": round(score_mean, 5),
-                "timing": f"CUDA events around the score kernel, {n_phase} live steps",
+                "algorithmic_bytes_per_launch": kernel_bytes, "ms_per_launch": round(score_mean, 5),
+                "timing": f"CUDA events around {what}, {n_phase} live steps",
                 "nominal_hbm_gbs": NOMINAL_HBM_GBS}
     step_bytes = k_bytes + moved_bytes
     step_achieved = step_bytes / (ms_per_step / 1e3) / 1e9
+    phases = {"query": round(statistics.mean(query_ms), 5), "score": round(score_mean, 5),
+              "select_compact": round(statistics.mean(evict_ms), 5)}
+    select_compact = {"kernel": "select_compact_kernel" if fused else "evict_kernel + move_kernel x2",
+                      "ms": round(statistics.mean(evict_ms), 5), "moved_bytes": moved_bytes,
+                      "achieved_moved_gbs": round(moved_bytes / (statistics.mean(evict_ms) / 1e3) / 1e9, 1)}
     step_roofline = {"bound": "hbm", "achieved": round(step_achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(step_achieved / peak, 4), "bytes_per_step": step_bytes,
-                     "moved_rows": moved, "phase_ms_serialised": {"query": round(statistics.mean(query_ms), 5),
-                                                       "score": round(score_mean, 5),
-                                                       "select_compact": round(statistics.mean(evict_ms), 5)}}
+                     "moved_rows": moved, "phase_ms_serialised": phases, "select_compact": select_compact}
 
     # ------------------------------------------------------------ e2e
     e2e = None
@@ -569,10 +586,12 @@ def run_ours(args, world, rank, local, dist):
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
                    "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
                    "launch": "CUDA graph replay of one captured step" if args.graph else "direct calls",
+                   "kernels": ("query_kernel, score kernel, select_compact_kernel" if fused else
+                               "query_kernel, score kernel, evict_kernel, move_kernel x2"),
                    "timing": "CUDA events around each tri_compress_step; kept-region restore and L2 flush "
                              "untimed; per-phase times from a separate live loop with phase events"},
         "roofline": roofline, "step_roofline": step_roofline,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": 5 * args.steps, "clocks": clk,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (3 if fused else 5) * args.steps, "clocks": clk,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
@@ -601,6 +620,7 @@ def run_decode(args, world, rank, local, dist, cfg):
     cache = tri.KvCache(wl.k_pool, wl.v_pool, wl.block_table, wl.seq_len, wl.cur_pos,
                         torch.zeros(1, dtype=torch.int32, device=dev), G)
     opt = tri.step_options(B, W, args.sinks, args.trigger)
+    fused = tri.tri_step_is_fused(cache, opt)
     ws = tri.alloc_workspace(cache, opt)
     fl = tri.FreeList.from_ids(wl.free_blocks, wl.num_blocks, dev)
     n_new = torch.full((S,), cfg.decode_append, dtype=torch.int32, device=dev)
@@ -665,6 +685,8 @@ def run_decode(args, world, rank, local, dist, cfg):
         "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "sequences": S,
                    "budget": B, "window": W, "append_per_round": cfg.decode_append,
                    "free_list": "device (tri_reserve_blocks pops, the step pushes; no host read of freed ids)",
+                   "kernels": ("query_kernel, score kernel, select_compact_kernel" if fused else
+                               "query_kernel, score kernel, evict_kernel, move_kernel x2"),
                    "timing": "CUDA events around each round's tri_compress_step_ex; appends untimed",
                    "rounds": rounds},
         "roofline": {"bound": "hbm", "achieved": round(all_bytes / (total_ms / 1e3) / 1e9, 1), "peak": peak,
@@ -680,7 +702,7 @@ def run_decode(args, world, rank, local, dist, cfg):
                                        "achieved": round(steady_bytes / (steady_ms / 1e3) / 1e9, 1),
                                        "frac": round(steady_bytes / (steady_ms / 1e3) / 1e9 / peak, 4)},
                      "achieved_k_read_first_round": rounds[0]["k_read_gbs"] if rounds else None},
-        "gpu_launches": 5 * cfg.decode_rounds, "clocks": clocks.summary(),
+        "gpu_launches": (3 if fused else 5) * cfg.decode_rounds, "clocks": clocks.summary(),
     }
     if rank == 0:
         print(json.dumps(out), flush=True)

@@ -443,6 +443,18 @@ tri_status tri_compress_step_ex(tri_kv_desc *desc, const float *qbar, const floa
                                 cudaStream_t stream);
 
 /*
+ * tri_step_is_fused - 1 if a step with these options (tri_compress_step,
+ * tri_compress_step_ex, tri_compress_step_distance) selects and compacts
+ * in one persistent kernel after its score pass, 0 if it runs selection,
+ * copy-out and move as separate kernels, -1 for an invalid descriptor or
+ * options.  The results are the same either way; only the launch sequence
+ * differs.  The persistent kernel serves every step (two CTAs per SM up to
+ * budget 4096, one above) unless the environment sets TRI_UNFUSED_STEP=1.
+ * Host-only, no CUDA work is queued.
+ */
+int tri_step_is_fused(const tri_kv_desc *desc, const tri_step_options *opt);
+
+/*
  * tri_reserve_blocks - grow sequences by n_new[s] slots each, taking the
  * paged blocks they newly need from the top of a device free list
  * ([GeoTrick] "Why Existing KV Cache Compression Breaks in Production": the

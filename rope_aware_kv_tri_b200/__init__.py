@@ -52,7 +52,7 @@ EXPORTS = (
     "tri_sync_status", "tri_status_string", "tri_workspace_size_ex", "tri_score_ex", "tri_select_topk_ex",
     "tri_compress_step_ex", "tri_reserve_blocks", "tri_distance_table", "tri_score_distance",
     "tri_compress_step_distance", "tri_selftest_bounded_wait", "tri_static_scratch_bytes",
-    "tri_check_stats",
+    "tri_check_stats", "tri_step_is_fused",
 )
 
 
@@ -168,6 +168,7 @@ def _load() -> ctypes.CDLL:
         "tri_selftest_bounded_wait": (I, [P, P, P]),
         "tri_static_scratch_bytes": (S, []),
         "tri_check_stats": (I, [P, P, P, I, I, I, P, P, P]),
+        "tri_step_is_fused": (I, [desc_p, ctypes.POINTER(TriStepOptions)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -426,6 +427,14 @@ def tri_compress_step_distance(cache: KvCache, table, slot_pos, opt: TriStepOpti
         _ptr(idx_out, torch.int32, "idx_out", allow_none=True),
         _ptr(workspace, torch.uint8, "workspace"), workspace.numel(), _events(events), _stream(stream))
     _check(code, "tri_compress_step_distance")
+
+
+def tri_step_is_fused(cache: KvCache, opt: TriStepOptions) -> bool:
+    """Whether the step with these options runs as the one fused kernel."""
+    r = int(library().tri_step_is_fused(cache.ref, ctypes.byref(opt)))
+    if r < 0:
+        raise TriError(TRI_ERR_INVALID, "tri_step_is_fused")
+    return r == 1
 
 
 def tri_check_stats(qbar, qabs, R, status, head_flags=None, stream=None) -> None:

@@ -20,8 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB_PATH = os.path.join(LIB_DIR, "libtriattn.so")
-SOURCES = ["tri_abi.cu", "calibrate.cu", "query.cu", "score.cu", "score_mma.cu", "evict.cu", "distance.cu", "tri_static_scratch.cu", "selftest.cu", "stats_check.cu"]
-HEADERS = ["tri_device.cuh", "tri_internal.h"]
+SOURCES = ["tri_abi.cu", "calibrate.cu", "query.cu", "score.cu", "score_mma.cu", "evict.cu", "distance.cu", "tri_static_scratch.cu", "selftest.cu", "stats_check.cu", "select_compact.cu"]
+HEADERS = ["tri_device.cuh", "tri_internal.h", "select_device.cuh", "score_device.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -89,6 +89,7 @@ __global__ void __launch_bounds__(kTableThreads) distance_table_kernel(const Dis
 // Block (u, chunk): slots [chunk*kDistChunk, ...) of unit u.
 __global__ void __launch_bounds__(kDistThreads) distance_score_kernel(const DistScoreParams p) {
     __shared__ uint32_t wlo[kDistThreads / 32], whi[kDistThreads / 32];
+    allow_next_grid();
     wait_prior_grid();
     const int u = blockIdx.x;
     const int LH = p.L * p.Hkv;

@@ -138,6 +138,7 @@ __device__ void plan_sequences(const QueryParams& p) {
         carry_items += tot_i;
         carry_freed += tot_f;
     }
+    if (p.fq_words && threadIdx.x < kQwWords) p.fq_words[threadIdx.x] = 0;   // select + compact unit counter
     if (p.plan_only && p.unit_kmin) {
         const int U = p.S * p.L * p.Hkv;
         for (int u = threadIdx.x; u < U; u += kQueryThreads) {
@@ -167,6 +168,7 @@ __device__ void plan_sequences(const QueryParams& p) {
 }
 
 __global__ void __launch_bounds__(kQueryThreads) query_kernel(const QueryParams p, int ctas_per_seq) {
+    allow_next_grid();
     const int n_query_ctas = p.S * ctas_per_seq;
     if ((int)blockIdx.x == n_query_ctas) {
         plan_sequences(p);

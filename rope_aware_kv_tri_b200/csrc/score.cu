@@ -42,6 +42,7 @@
 // G partial sums are reduced with a butterfly that halves the live heads at
 // each step (a reduce-scatter over the key's lanes), then the lanes holding
 // different heads' totals exchange their maximum.
+#include "score_device.cuh"
 #include "tri_device.cuh"
 #include "tri_internal.h"
 
@@ -72,25 +73,6 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
         }
     }
     return false;
-}
-
-// This lane's part of a key score: 8 bands (4 adjacent pairs) of the real
-// half a and the imaginary half b, with packed-pair fp32 arithmetic.
-__device__ __forceinline__ float key_score(const uint4 a, const uint4 b, const float2 (&qr)[4],
-                                           const float2 (&qi)[4], const float2 (&ww)[4]) {
-    const uint32_t av[4] = {a.x, a.y, a.z, a.w};
-    const uint32_t bv[4] = {b.x, b.y, b.z, b.w};
-    float2 dot = make_float2(0.f, 0.f), nrm = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        const float2 r = make_float2(bf16_lo(av[j]), bf16_hi(av[j]));
-        const float2 i = make_float2(bf16_lo(bv[j]), bf16_hi(bv[j]));
-        dot = ffma2(qr[j], r, dot);
-        dot = ffma2(qi[j], i, dot);
-        const float2 sq = ffma2(r, r, fmul2(i, i));
-        nrm = ffma2(ww[j], make_float2(sqrt_fast(sq.x), sqrt_fast(sq.y)), nrm);
-    }
-    return (dot.x + dot.y) + (nrm.x + nrm.y);
 }
 
 // ---- max over the group -------------------------------------------------
@@ -283,17 +265,7 @@ __device__ void consume(const ScoreParams& p, int warp, int lane, const uint8_t*
             const int unit = m.unit0 + hig;
             if (unit != cur_unit) {
                 flush_range();
-                const float4* qe = reinterpret_cast<const float4*>(p.qeff + (int64_t)unit * kHeadDim);
-                const float4* we = reinterpret_cast<const float4*>(p.wts + (int64_t)unit * kBands);
-                const float4 x0 = qe[2 * sub], x1 = qe[2 * sub + 1];
-                const float4 y0 = qe[16 + 2 * sub], y1 = qe[16 + 2 * sub + 1];
-                const float4 z0 = we[2 * sub], z1 = we[2 * sub + 1];
-                qr[0] = make_float2(x0.x, x0.y); qr[1] = make_float2(x0.z, x0.w);
-                qr[2] = make_float2(x1.x, x1.y); qr[3] = make_float2(x1.z, x1.w);
-                qi[0] = make_float2(y0.x, y0.y); qi[1] = make_float2(y0.z, y0.w);
-                qi[2] = make_float2(y1.x, y1.y); qi[3] = make_float2(y1.z, y1.w);
-                ww[0] = make_float2(z0.x, z0.y); ww[1] = make_float2(z0.z, z0.w);
-                ww[2] = make_float2(z1.x, z1.y); ww[3] = make_float2(z1.z, z1.w);
+                load_key_coefficients(p.qeff, p.wts, unit, sub, qr, qi, ww);
                 cur_unit = unit;
             }
             const uint8_t* tile = tiles + (size_t)slot * stage_bytes + (size_t)hig * kTileBytes;
@@ -433,6 +405,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
         fence_mbar_init();
     }
     __syncthreads();
+    allow_next_grid();
     wait_prior_grid();          // the folded queries and the plan come from query_kernel
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == kConsumerWarps) {

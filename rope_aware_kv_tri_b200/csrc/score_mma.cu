@@ -614,6 +614,7 @@ __global__ void __launch_bounds__(kMmaThreads, 1) score_mma_kernel(const __grid_
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *sm.tmem_slot;
+    allow_next_grid();
     wait_prior_grid();          // effective queries and the plan come from query_kernel
 
     if (warp == kProducerWarp) {

@@ -7,6 +7,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstdlib>
 #include <mutex>
 
 #include "tri_attention.h"
@@ -21,7 +22,7 @@ constexpr size_t kWsAlign = 256;
 size_t align_up(size_t x) { return (x + kWsAlign - 1) & ~(kWsAlign - 1); }
 
 struct WsLayout {
-    size_t qeff, wts, len_ws, item_off, freed_off, kmin, kmax, scores, idx, words, info, owner, scratch, total;
+    size_t qeff, wts, len_ws, item_off, freed_off, kmin, kmax, scores, idx, words, info, owner, scratch, fq, total;
     int scratch_rows;
 };
 
@@ -56,6 +57,8 @@ WsLayout ws_layout(const tri_kv_desc* d, int budget, bool per_head = false) {
     w.info = off;      off = align_up(off + U * 4 * sizeof(int32_t) * per_unit);
     w.owner = off;     off = align_up(off + (size_t)w.scratch_rows * 2 * sizeof(int32_t));
     w.scratch = off;   off = align_up(off + (size_t)w.scratch_rows * 2 * kHeadDim * 2);
+    // select + compact kernel: its unit counter
+    w.fq = off;        off = align_up(off + (size_t)kQwWords * sizeof(int32_t) * per_unit);
     w.total = off;
     return w;
 }
@@ -124,6 +127,18 @@ tri_status check_options(const tri_step_options* o, int G) {
 
 int effective_trigger(const tri_step_options& o) { return o.trigger > o.budget ? o.trigger : o.budget; }
 
+// TRI_UNFUSED_STEP=1 in the environment makes a step run its selection and
+// compaction as separate kernels (selection, copy-out, move) even where the
+// persistent select + compact kernel applies; both give the same results.
+// Read once.
+bool unfused_step_forced() {
+    static const bool forced = [] {
+        const char* v = std::getenv("TRI_UNFUSED_STEP");
+        return v != nullptr && v[0] == '1';
+    }();
+    return forced;
+}
+
 tri_status check_free_list(const tri_free_list* fl) {
     if (fl == nullptr) return TRI_OK;
     if (!fl->ids || !fl->count || fl->capacity < 0 || !aligned(fl->ids, 4) || !aligned(fl->count, 4))
@@ -132,6 +147,10 @@ tri_status check_free_list(const tri_free_list* fl) {
 }
 
 tri_status cuda_status(cudaError_t e) { return e == cudaSuccess ? TRI_OK : TRI_ERR_CUDA; }
+
+// Whether a step with this budget selects and compacts in the persistent
+// select + compact kernel (select_compact.cu).
+bool persistent_compaction(int budget) { return !unfused_step_forced() && select_compact_supported(budget); }
 
 int device_sm_count() {
     static std::mutex mu;
@@ -262,6 +281,7 @@ void set_step_plan(QueryParams& q, const tri_kv_desc* desc, uint8_t* ws, const W
         q.fl_capacity = free_list->capacity;
         q.fl_base = reinterpret_cast<int32_t*>(ws + w.words) + 2;
     }
+    if (persistent_compaction(budget)) q.fq_words = reinterpret_cast<int32_t*>(ws + w.fq);
 }
 
 // The selection and compaction launches of a step, after its scores are in
@@ -270,6 +290,40 @@ tri_status select_and_compact(const tri_kv_desc* desc, uint8_t* ws, const WsLayo
                               int trigger, const tri_free_list* free_list, int32_t* freed_ids, int32_t* idx_out,
                               int32_t* slot_pos, bool pdl, cudaStream_t stream, const int32_t* veto = nullptr) {
     const int budget = opt.budget;
+    if (persistent_compaction(budget)) {
+        SelectCompactParams c{};
+        c.k_pool = static_cast<uint8_t*>(desc->k_pool);
+        c.v_pool = static_cast<uint8_t*>(desc->v_pool);
+        c.block_table = desc->block_table;
+        c.len_ws = reinterpret_cast<const int32_t*>(ws + w.len_ws);
+        c.scores = reinterpret_cast<const float*>(ws + w.scores);
+        c.score_stride = (int64_t)desc->max_blocks * kBlockRows;
+        c.unit_kmin = reinterpret_cast<const uint32_t*>(ws + w.kmin);
+        c.unit_kmax = reinterpret_cast<const uint32_t*>(ws + w.kmax);
+        c.status = desc->status;
+        c.L = desc->L;
+        c.Hkv = desc->Hkv;
+        c.num_blocks = desc->num_blocks;
+        c.S = desc->S;
+        c.max_blocks = desc->max_blocks;
+        c.budget = budget;
+        c.window = opt.window;
+        c.sinks = opt.sinks;
+        c.trigger = trigger;
+        c.idx_copy = idx_out;
+        c.seq_len_out = desc->seq_len;
+        c.freed_off = reinterpret_cast<const int32_t*>(ws + w.freed_off);
+        c.freed_ids = freed_ids;
+        if (free_list) {
+            c.fl_ids = free_list->ids;
+            c.fl_base = reinterpret_cast<const int32_t*>(ws + w.words) + 2;
+        }
+        c.slot_pos = slot_pos;
+        c.pos_stride = (int64_t)desc->max_blocks * kBlockRows;
+        c.abort_word = veto;
+        c.qwords = reinterpret_cast<int32_t*>(ws + w.fq);
+        return cuda_status(launch_select_compact(c, device_sm_count(), stream, pdl));
+    }
     EvictParams e = make_evict_params(desc);
     e.scores = reinterpret_cast<const float*>(ws + w.scores);
     e.unit_kmin = reinterpret_cast<const uint32_t*>(ws + w.kmin);
@@ -567,6 +621,11 @@ tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const floa
         return st;
     if (events) record(events->after_evict, stream);
     return TRI_OK;
+}
+
+int tri_step_is_fused(const tri_kv_desc* desc, const tri_step_options* opt) {
+    if (check_desc(desc) != TRI_OK || check_options(opt, desc->G) != TRI_OK) return -1;
+    return persistent_compaction(opt->budget) ? 1 : 0;
 }
 
 tri_status tri_check_stats(const float* qbar, const float* qabs, const float* R, int L, int Hq, int D,

@@ -52,6 +52,13 @@ __device__ __forceinline__ void st_release_gpu(int32_t* p, int v) {
 // launched without the programmatic-serialization attribute).
 __device__ __forceinline__ void wait_prior_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Programmatic dependent launch: let the next kernel in the stream (launched
+// with the programmatic-serialization attribute) be scheduled as soon as
+// every CTA of this grid has executed this or exited.  It still waits for
+// this grid to complete (wait_prior_grid) before reading what it wrote, so
+// only its launch latency overlaps this grid.
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

@@ -67,6 +67,7 @@ struct QueryParams {
     int fl_capacity;
     int32_t* fl_base;         // [1] out: first list entry of this step's ids, -1 if no room
     const int32_t* abort_word; // non-zero: the statistics check vetoed the step (plan nothing), or null
+    int32_t* fq_words;         // select + compact: queue words to zero (kQwWords), or null
     int32_t* status;
 };
 cudaError_t launch_query(const QueryParams& p, cudaStream_t stream);
@@ -141,6 +142,39 @@ struct EvictParams {
     const int32_t* abort_word; // non-zero: the step was vetoed, touch nothing; or null
 };
 cudaError_t launch_evict(const EvictParams& p, cudaStream_t stream, bool pdl = false);
+
+// ------------------------------ select + compact (select_compact.cu)
+// Selection and compaction of a step's units in one persistent kernel,
+// after the score pass; used by every step variant whose budget fits.
+// Queue words (workspace, zeroed by the plan CTA):
+constexpr int kQwClaim = 0;     // next unit to take
+constexpr int kQwWords = 8;
+
+struct SelectCompactParams {
+    uint8_t* k_pool;
+    uint8_t* v_pool;
+    const int32_t* block_table;
+    const int32_t* len_ws;     // [S] lengths the step works from
+    const float* scores;
+    int64_t score_stride;
+    const uint32_t* unit_kmin; // [U] score-key range of each unit
+    const uint32_t* unit_kmax;
+    int32_t* status;
+    int L, Hkv, num_blocks, S, max_blocks;
+    int budget, window, sinks, trigger;
+    int32_t* idx_copy;         // [U][budget] kept slots out, or null
+    int32_t* seq_len_out;
+    const int32_t* freed_off;
+    int32_t* freed_ids;        // or null
+    int32_t* fl_ids;           // free list entries, or null
+    const int32_t* fl_base;
+    int32_t* slot_pos;         // [U][pos_stride] positions compacted with the rows, or null
+    int64_t pos_stride;
+    const int32_t* abort_word; // non-zero: the step was vetoed; or null
+    int32_t* qwords;           // [kQwWords]
+};
+bool select_compact_supported(int budget);
+cudaError_t launch_select_compact(const SelectCompactParams& p, int num_sms, cudaStream_t stream, bool pdl);
 
 // Phase 2 of the compaction for all units (after launch_evict's phase 1).
 struct MoveParams {
