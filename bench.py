@@ -18,8 +18,10 @@ whole step against the measured B200 copy bandwidth.
 GPU, NCCL); under torchrun WORLD_SIZE must equal --gpus.
 
 Timing: each timed step restores the kept region of the cache and flushes L2
-(256 MiB write) outside CUDA events that bracket only the tri_compress_step
-launches; the K/V pools (4.3 GB) are larger than L2 as well.  The timed loop
+outside CUDA events that bracket only the tri_compress_step launches: a
+256 MiB buffer is written, then (default --l2-flush clean) another 256 MiB is
+read, so the write's dirty lines reach DRAM before the step instead of during
+its first kernels.  The K/V pools (4.3 GB) are larger than L2 as well.  The timed loop
 is bracketed by a barrier and a device synchronize; the step time is the
 maximum over ranks.  Ranks run independent caches (weak scaling: units
 shard across GPUs with no data-path collective).
@@ -71,12 +73,41 @@ def parse_args(argv=None):
                     help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--phases", action="store_true",
                     help="decode loop: time each round's phases with library events (serialises launches)")
+    ap.add_argument("--l2-flush", choices=["clean", "dirty"], default="clean",
+                    help="between timed steps write a buffer larger than L2, then (clean) read a second one so "
+                         "that the write's dirty lines are written back before the step, or (dirty) not")
     ap.add_argument("--layers", type=int, default=0,
                     help="override the layer count (small profiling cases of the same kernels)")
     return ap.parse_args(argv)
 
 
 # ----------------------------------------------------------------- helpers
+
+class L2Flush:
+    """Evicts the step's data from L2 between timed steps: writes a buffer
+    larger than L2; in "clean" mode then reads a second one, so the write's
+    dirty lines are written back before the timed step rather than during
+    its first kernels (the state after kernels that only read, such as
+    attention over the cache)."""
+
+    def __init__(self, mode: str, dev):
+        import torch
+        self.mode = mode
+        self.buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.buf2 = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev) if mode == "clean" else None
+
+    def __call__(self):
+        self.buf.zero_()
+        if self.buf2 is not None:
+            self.buf2.amax()
+
+    def describe(self) -> str:
+        mib = L2_FLUSH_BYTES >> 20
+        if self.mode == "clean":
+            return (f"K/V pools larger than L2; between timed steps {mib} MiB written, then another {mib} MiB "
+                    "read (L2 holds no step data and no dirty lines)")
+        return f"K/V pools larger than L2; {mib} MiB written between timed steps (L2 left dirty)"
+
 
 def measured_peak():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -415,7 +446,7 @@ def run_ours(args, world, rank, local, dist):
     save_k = wl.k_pool[:, rblocks].clone()
     save_v = wl.v_pool[:, rblocks].clone()
     save_len = wl.seq_len.clone()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(args.l2_flush, dev)
     table_ms = None
     if distance:
         # one-time table of the centres (untimed, like the calibration)
@@ -438,7 +469,7 @@ def run_ours(args, world, rank, local, dist):
         wl.seq_len.copy_(save_len)
         if distance:
             slot_pos[..., :B] = save_pos
-        flush.zero_()
+        flush()
 
     def step(events=None, idx_out=None):
         if distance:
@@ -536,13 +567,14 @@ def run_ours(args, world, rank, local, dist):
                                                        else "score_kernel")
     kernel_bytes = k_bytes
     what = "the score kernel"
-    achieved = kernel_bytes / (score_mean / 1e3) / 1e9
+    kernel_ms = score_mean
+    achieved = kernel_bytes / (kernel_ms / 1e3) / 1e9
     tpl = recorded_traffic_per_launch(kernel, keys_per_step, moved) if not variant and not distance else None
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                 "frac": round(achieved / peak, 4), "traffic": tpl, "kernel": kernel,
                 "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_kind == "measured" else "fallback 6650 GB/s",
-                "algorithmic_bytes_per_launch": kernel_bytes, "ms_per_launch": round(score_mean, 5),
+                "algorithmic_bytes_per_launch": kernel_bytes, "ms_per_launch": round(kernel_ms, 5),
                 "timing": f"CUDA events around {what}, {n_phase} live steps",
                 "nominal_hbm_gbs": NOMINAL_HBM_GBS}
     step_bytes = k_bytes + moved_bytes
@@ -584,17 +616,30 @@ def run_ours(args, world, rank, local, dist):
                                    f"counts all-reduced (equal on every rank: {freed_same})" if heads_mode else
                                    f"units sharded: one independent cache per GPU x{world}"),
                    "input_dtype": "bf16 K/V, fp32 arithmetic",
-                   "l2": "K/V pools larger than L2; 256 MiB L2 flush between timed steps",
+                   "l2": flush.describe(),
                    "launch": "CUDA graph replay of one captured step" if args.graph else "direct calls",
-                   "kernels": ("query_kernel, score kernel, select_compact_kernel" if fused else
-                               "query_kernel, score kernel, evict_kernel, move_kernel x2"),
+                   "kernels": kernel_list(fused, distance),
                    "timing": "CUDA events around each tri_compress_step; kept-region restore and L2 flush "
                              "untimed; per-phase times from a separate live loop with phase events"},
         "roofline": roofline, "step_roofline": step_roofline,
-        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": (3 if fused else 5) * args.steps, "clocks": clk,
+        "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches_per_step(fused) * args.steps, "clocks": clk,
     }
     if rank == 0:
         print(json.dumps(out), flush=True)
+
+
+def kernel_list(fused: bool, distance: bool) -> str:
+    """The kernels one step launches, in order."""
+    first = "query_kernel (plan only)" if distance else "query_kernel"
+    middle = "distance_score_kernel" if distance else "score kernel"
+    last = "select_compact_kernel" if fused else "evict_kernel, move_kernel x2"
+    return f"{first}, {middle}, {last}"
+
+
+def launches_per_step(fused: bool) -> int:
+    """How many of the library's kernels one step launches (the same count
+    for both score modes: the plan, one scoring kernel, then compaction)."""
+    return 3 if fused else 5
 
 
 def run_decode(args, world, rank, local, dist, cfg):
@@ -624,7 +669,7 @@ def run_decode(args, world, rank, local, dist, cfg):
     ws = tri.alloc_workspace(cache, opt)
     fl = tri.FreeList.from_ids(wl.free_blocks, wl.num_blocks, dev)
     n_new = torch.full((S,), cfg.decode_append, dtype=torch.int32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(args.l2_flush, dev)
     # kept slots of every unit (an optional output of the step), to count the
     # rows each round moves once the round is over
     idx = torch.empty(S, L, Hkv, B, dtype=torch.int32, device=dev)
@@ -642,7 +687,7 @@ def run_decode(args, world, rank, local, dist, cfg):
         wl.cur_pos += cfg.decode_append
         lens = wl.seq_len.tolist()
         free_before = int(fl.count.item())
-        flush.zero_()
+        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         pev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if args.phases else None
         torch.cuda.synchronize(dev)
@@ -685,8 +730,8 @@ def run_decode(args, world, rank, local, dist, cfg):
         "config": {"workload": cfg.name, "L": L, "Hkv": Hkv, "G": G, "D": 128, "sequences": S,
                    "budget": B, "window": W, "append_per_round": cfg.decode_append,
                    "free_list": "device (tri_reserve_blocks pops, the step pushes; no host read of freed ids)",
-                   "kernels": ("query_kernel, score kernel, select_compact_kernel" if fused else
-                               "query_kernel, score kernel, evict_kernel, move_kernel x2"),
+                   "l2": flush.describe(),
+                   "kernels": kernel_list(fused, False),
                    "timing": "CUDA events around each round's tri_compress_step_ex; appends untimed",
                    "rounds": rounds},
         "roofline": {"bound": "hbm", "achieved": round(all_bytes / (total_ms / 1e3) / 1e9, 1), "peak": peak,
@@ -702,7 +747,7 @@ def run_decode(args, world, rank, local, dist, cfg):
                                        "achieved": round(steady_bytes / (steady_ms / 1e3) / 1e9, 1),
                                        "frac": round(steady_bytes / (steady_ms / 1e3) / 1e9 / peak, 4)},
                      "achieved_k_read_first_round": rounds[0]["k_read_gbs"] if rounds else None},
-        "gpu_launches": (3 if fused else 5) * cfg.decode_rounds, "clocks": clocks.summary(),
+        "gpu_launches": launches_per_step(fused) * cfg.decode_rounds, "clocks": clocks.summary(),
     }
     if rank == 0:
         print(json.dumps(out), flush=True)

@@ -15,8 +15,9 @@ Both paths are also checked against the oracle elsewhere; this file pins
 them to each other on shapes that stress the persistent kernel:
 ragged lengths, a shuffled table, several sequences (one short enough to be
 left alone), sinks and a trigger, a free list, budgets 1024 to 8192 (one CTA
-per SM above 4096), the maximum over the group, and the headline 32-layer x
-8-head T = 32768 shape.
+per SM above 4096), the maximum over the group, the headline 32-layer x
+8-head T = 32768 shape, and the distance-table step (where the kernel also
+carries each unit's slot positions with its rows).
 """
 
 import json
@@ -40,6 +41,8 @@ CASES = {
     "budget_8192_max": dict(base="l64h8g8_4x64k", L=2, lens=[9000, 30000], budget=8192, window=128, sinks=0,
                             trigger=0, n_samples=256, aggregate="max"),
     "headline_32L_8H_T32768": dict(base="l32h8_t32k", sinks=0, trigger=0),
+    "distance_table_step": dict(base="l32h8_t32k", L=4, lens=[32768, 9000, 1500], budget=2048, window=128, sinks=3,
+                                trigger=0, n_samples=256, distance=True),
 }
 
 
@@ -55,6 +58,7 @@ def run_case(name: str, out_path: str) -> None:
     base = spec.pop("base")
     sinks, trigger = spec.pop("sinks"), spec.pop("trigger")
     agg = tri.TRI_AGG_MAX if spec.pop("aggregate", "mean") == "max" else tri.TRI_AGG_MEAN
+    distance = spec.pop("distance", False)
     cfg = CONFIGS[base].replace(**spec)
     dev = "cuda"
     wl = make_workload(cfg, device=dev, seed=11)
@@ -68,8 +72,19 @@ def run_case(name: str, out_path: str) -> None:
     count = torch.full((1,), -7, dtype=torch.int32, device=dev)
     idx = torch.full((S, L, Hkv, B), -7, dtype=torch.int32, device=dev)
     lens = wl.seq_len.cpu().tolist()
-    tri.tri_compress_step_ex(cache, *stats, cfg.base, wl.deltas, opt, ws, free_list=fl, freed_ids=freed,
-                             freed_count=count, idx_out=idx)
+    slot_pos = None
+    if distance:
+        # the distance-table step: scores from a table of the centres, positions carried with the rows
+        max_dist = int(wl.cur_pos.max().item()) + 1
+        table = torch.empty(L, Hkv, max_dist + 1, device=dev)
+        tri.tri_distance_table(stats[0], wl.key_centres.float().contiguous(), cfg.base, wl.deltas, tri.TRI_AGG_MEAN,
+                               table)
+        slot_pos = torch.arange(wl.max_blocks * 16, dtype=torch.int32, device=dev).repeat(S, L, Hkv, 1).contiguous()
+        tri.tri_compress_step_distance(cache, table, slot_pos, opt, ws, free_list=fl, freed_ids=freed,
+                                       freed_count=count, idx_out=idx)
+    else:
+        tri.tri_compress_step_ex(cache, *stats, cfg.base, wl.deltas, opt, ws, free_list=fl, freed_ids=freed,
+                                 freed_count=count, idx_out=idx)
     code = tri.tri_sync_status(cache.status)
     n = int(count.item())
     table = wl.block_table.cpu().tolist()
@@ -89,7 +104,8 @@ def run_case(name: str, out_path: str) -> None:
                 if (s, l, h) in ((0, 0, 0), (S - 1, L - 1, Hkv - 1), (S // 2, L // 2, Hkv // 2)):
                     sample[f"{s}.{l}.{h}"] = unit_rows(wl.k_pool, table[s], lens[s], l, h).view(torch.int16).cpu()
     torch.save({"code": code, "idx": idx.cpu(), "freed": freed[:n].cpu(), "len": wl.seq_len.cpu(),
-                "fl": fl.contents(), "sums": sums, "sample": sample}, out_path)
+                "fl": fl.contents(), "sums": sums, "sample": sample,
+                "pos": slot_pos.cpu() if slot_pos is not None else None}, out_path)
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -120,3 +136,5 @@ def test_persistent_compaction_equals_separate_kernels(name, tmp_path):
     assert not bad, f"{len(bad)} units' rows differ, e.g. {bad[:4]}"
     for k in a["sample"]:
         assert torch.equal(a["sample"][k], b["sample"][k]), k
+    if a["pos"] is not None:
+        assert torch.equal(a["pos"], b["pos"]), "carried positions differ"
