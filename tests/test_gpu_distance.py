@@ -7,7 +7,9 @@
 * tri_compress_step_distance on a table made on the host (the oracle's, in
   fp32) that both sides use: selection, compaction, freed blocks and the
   compacted slot positions are bit-exact, for caches whose slots still equal
-  their positions and for caches compacted before (positions with gaps).
+  their positions and for caches compacted before (positions with gaps);
+* the same step at the benchmark's full size (32 layers x 8 KV heads,
+  T = 32768), on the table tri_distance_table builds.
 """
 
 import numpy as np
@@ -16,7 +18,7 @@ import torch
 
 import oracle
 import rope_aware_kv_tri_b200 as tri
-from tests.gpu_helpers import cache_of, expected_pools_after, freed_expected
+from tests.gpu_helpers import cache_of, expected_pools_after, freed_expected, gpu_stats
 from tests.test_gpu_parity import SMALL
 from workload import make_workload
 
@@ -147,3 +149,68 @@ def test_compress_step_distance_matches_oracle(sinks, trigger):
     assert torch.equal(wl.v_pool.view(torch.int16), ev.view(torch.int16))
     assert np.array_equal(wl.k_pool.view(torch.int16).cpu().numpy(), ref["k_pool"])
     assert np.array_equal(wl.v_pool.view(torch.int16).cpu().numpy(), ref["v_pool"])
+
+
+def test_full_size_distance_step_32L_8H_T32768():
+    """The benchmark's distance-table step at its full size (32 layers x 8 KV
+    heads, one sequence of 32768 slots, B = 2048, W = 128) in the launch
+    configuration bench.py times: the table built by tri_distance_table
+    (sampled heads against the oracle's table), then one
+    tri_compress_step_distance.  Every unit's kept slots, every row of both
+    pools and every carried position are checked; sampled units' kept slots
+    equal the oracle's selection on the same table values, bit for bit."""
+    from workload import CONFIGS
+    wl = make_workload(CONFIGS["l32h8_t32k"], device=DEV, seed=0)
+    cfg = wl.cfg
+    S, L, Hkv, G = cfg.S, cfg.L, cfg.Hkv, cfg.G
+    budget, window = cfg.budget, cfg.window
+    qbar = gpu_stats(wl)[0]
+    kbar = wl.key_centres.float().contiguous()
+    max_dist = int(wl.cur_pos.max().item()) + 1
+    table = torch.empty(L, Hkv, max_dist + 1, device=DEV)
+    tri.tri_distance_table(qbar, kbar, cfg.base, wl.deltas, tri.TRI_AGG_MEAN, table)
+    torch.cuda.synchronize()
+    tab = table.cpu().numpy()
+    for l, h in ((0, 0), (L - 1, Hkv - 1)):
+        ref = oracle.distance_table(qbar[l, h * G:(h + 1) * G].double().cpu().numpy(),
+                                    kbar[l, h].double().cpu().numpy(), wl.deltas, cfg.base, max_dist)
+        scale = float(np.max(np.abs(ref)))
+        err = np.abs(tab[l, h].astype(np.float64) - ref)
+        assert np.all(err <= 1e-6 * np.abs(ref) + 1e-7 * scale), float((err / scale).max())
+    lens = wl.seq_len.cpu().tolist()
+    kept = [min(n, budget) for n in lens]
+    max_len = wl.max_blocks * 16
+    pos0 = torch.arange(max_len, dtype=torch.int32, device=DEV).repeat(S, L, Hkv, 1).contiguous()
+    gpos = pos0.clone()
+    pk, pv = wl.k_pool.clone(), wl.v_pool.clone()
+    cache = cache_of(wl)
+    opt = tri.step_options(budget, window)
+    ws = tri.alloc_workspace(cache, opt)
+    freed = torch.full((S * wl.max_blocks,), -7, dtype=torch.int32, device=DEV)
+    count = torch.full((1,), -7, dtype=torch.int32, device=DEV)
+    idx = torch.full((S, L, Hkv, budget), -7, dtype=torch.int32, device=DEV)
+    tri.tri_compress_step_distance(cache, table, gpos, opt, ws, freed_ids=freed, freed_count=count, idx_out=idx)
+    assert tri.tri_sync_status(cache.status) == tri.TRI_OK
+    assert wl.seq_len.cpu().tolist() == kept
+    assert freed[:int(count.item())].cpu().tolist() == freed_expected(wl.block_table, lens, kept)
+    ek, ev = expected_pools_after(pk, pv, wl.block_table, lens, idx, kept)
+    del pk, pv
+    assert torch.equal(wl.k_pool.view(torch.int16), ek.view(torch.int16))
+    assert torch.equal(wl.v_pool.view(torch.int16), ev.view(torch.int16))
+    del ek, ev
+    # positions travel with their rows; slots past the kept ones keep theirs
+    assert torch.equal(gpos[..., :budget], torch.gather(pos0, -1, idx.long()))
+    assert torch.equal(gpos[..., budget:], pos0[..., budget:])
+    # every unit: ascending, window kept; sampled units: the oracle's selection
+    assert torch.all(idx[..., 1:] > idx[..., :-1])
+    cand = lens[0] - window
+    assert torch.all(idx[..., budget - window:] == torch.arange(cand, lens[0], device=DEV, dtype=torch.int32))
+    p = wl.cur_pos.cpu().tolist()
+    rng = np.random.default_rng(1)
+    units = [(0, 0, 0), (S - 1, L - 1, Hkv - 1)] + [(0, int(rng.integers(L)), int(rng.integers(Hkv)))
+                                                    for _ in range(4)]
+    for s, l, h in units:
+        n = lens[s]
+        scores = oracle.distance_scores(tab[l, h].astype(np.float64), p[s], np.arange(n))
+        want = oracle.select(scores, n, budget, window)
+        assert np.array_equal(idx[s, l, h].cpu().numpy(), want), (s, l, h)
