@@ -296,16 +296,19 @@ __device__ __forceinline__ float key_value(uint32_t key) {
     return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
-// Linear bucket of score x in [lo, lo + (kLinBins-1)/scale]; monotone in x.
-__device__ __forceinline__ int lin_bucket(float x, float lo, float scale) {
+// Linear bucket of score x in [lo, lo + (nb-1)/scale] (nb buckets); monotone in x.
+__device__ __forceinline__ int lin_bucket(float x, float lo, float scale, int nb = kLinBins) {
     const int b = (int)((x - lo) * scale);
-    return b < 0 ? 0 : (b > kLinBins - 1 ? kLinBins - 1 : b);
+    return b < 0 ? 0 : (b > nb - 1 ? nb - 1 : b);
 }
 
 // Emit the set bits of `bits` (nwords words, slot 32w + b) into sidx in
 // ascending order, at most `take` of them.  Each warp takes a contiguous run
-// of words; lane i tests bit i of the warp's current word, so the warp writes
-// a whole word per step whatever its population.
+// of words.  A dense run (more than a quarter of its bits set) is walked a
+// word per step, lane i testing bit i, so every lane stores at once; a
+// sparse run is walked 64 words per step, lane i owning words 2i and 2i + 1:
+// a warp scan of their bit counts gives each lane its first output slot and
+// the lane stores its own set bits in order.
 template <int NT>
 __device__ void emit_kept(const uint32_t* bits, int nwords, int take, int* sidx, EvictSmem<NT>& sm) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -318,12 +321,33 @@ __device__ void emit_kept(const uint32_t* bits, int nwords, int take, int* sidx,
     sel_sync<NT>();
     int base = 0;
     for (int k = 0; k < warp; ++k) base += sm.warp_a[k];
-    const uint32_t lt = lanemask_lt();
-    for (int w = w0; w < w1; ++w) {
-        const uint32_t kw = bits[w];
-        const int pos = base + __popc(kw & lt);
-        if (((kw >> lane) & 1u) && pos < take) sidx[pos] = w * 32 + lane;
-        base += __popc(kw);
+    if (4 * cnt > 32 * (w1 - w0)) {
+        const uint32_t lt = lanemask_lt();
+        for (int w = w0; w < w1; ++w) {
+            const uint32_t kw = bits[w];
+            const int pos = base + __popc(kw & lt);
+            if (((kw >> lane) & 1u) && pos < take) sidx[pos] = w * 32 + lane;
+            base += __popc(kw);
+        }
+    } else {
+        for (int c0 = w0; c0 < w1; c0 += 64) {
+            const int wa = c0 + 2 * lane;
+            uint32_t a = wa < w1 ? bits[wa] : 0u;
+            uint32_t b = wa + 1 < w1 ? bits[wa + 1] : 0u;
+            const int n = __popc(a) + __popc(b);
+            int incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            int pos = base + incl - n;
+            for (; a; a &= a - 1u, ++pos)
+                if (pos < take) sidx[pos] = wa * 32 + (__ffs(a) - 1);
+            for (; b; b &= b - 1u, ++pos)
+                if (pos < take) sidx[pos] = (wa + 1) * 32 + (__ffs(b) - 1);
+            base += __shfl_sync(0xffffffffu, incl, 31);
+        }
     }
     sel_sync<NT>();
 }
@@ -401,11 +425,16 @@ __device__ void finish_from_list(const uint32_t* list_key, const int* list_slot,
 // above the cut's and the cut bucket's slots then come from shared memory,
 // and only the (few) cut-bucket scores are read again.
 template <int NT>
-__device__ bool select_one_pass(const float* __restrict__ sc, int cand, int first, int take, float lo, float scale,
+__device__ bool select_one_pass(const float* __restrict__ sc, int cand, int first, int take, float lo, float span,
                                 int* sidx, EvictSmem<NT>& sm) {
+    // about 4 candidates per bucket at most, 512 to kLinBins buckets: a short
+    // unit zeroes and scans fewer buckets
+    int nb = 512;
+    while (nb < kLinBins && 4 * nb < cand) nb <<= 1;
+    const float scale = (float)(nb - 1) / span;
     OnePassScratch& o = sm.u.sel.one;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < kLinBins; i += NT) o.hist[i] = 0;
+    for (int i = threadIdx.x; i < nb; i += NT) o.hist[i] = 0;
     sel_sync<NT>();
     const int nvec = cand >> 2;
     const float4* v4 = reinterpret_cast<const float4*>(sc);
@@ -420,8 +449,8 @@ __device__ bool select_one_pass(const float* __restrict__ sc, int cand, int firs
         for (int k = 0; k < kUnroll; ++k) {
             const int v = v0 + k * NT;
             if (v < nvec) {
-                const int b0 = lin_bucket(x[k].x, lo, scale), b1 = lin_bucket(x[k].y, lo, scale);
-                const int b2 = lin_bucket(x[k].z, lo, scale), b3 = lin_bucket(x[k].w, lo, scale);
+                const int b0 = lin_bucket(x[k].x, lo, scale, nb), b1 = lin_bucket(x[k].y, lo, scale, nb);
+                const int b2 = lin_bucket(x[k].z, lo, scale, nb), b3 = lin_bucket(x[k].w, lo, scale, nb);
                 *reinterpret_cast<uint2*>(&o.code[4 * v]) =
                     make_uint2((uint32_t)b0 | ((uint32_t)b1 << 16), (uint32_t)b2 | ((uint32_t)b3 << 16));
                 if (4 * v >= first) {
@@ -440,37 +469,56 @@ __device__ bool select_one_pass(const float* __restrict__ sc, int cand, int firs
         }
     }
     for (int t = 4 * nvec + threadIdx.x; t < cand; t += NT) {
-        const int b = lin_bucket(__ldcg(sc + t), lo, scale);
+        const int b = lin_bucket(__ldcg(sc + t), lo, scale, nb);
         o.code[t] = (uint16_t)b;
         if (t >= first) atomicAdd(&o.hist[b], 1);
     }
     sel_sync<NT>();
     int rem = take;
-    const int bstar = pick_bin<NT>(o.hist, kLinBins, rem, sm);
+    const int bstar = pick_bin<NT>(o.hist, nb, rem, sm);
     if (o.hist[bstar] > kOneListCap) return false;
     const int nwords = (cand + 31) / 32;
     for (int w = threadIdx.x; w < nwords; w += NT) o.eq_bits[w] = 0u;
     if (threadIdx.x == 0) sm.n_list = 0;
     sel_sync<NT>();
-    // 8 buckets per 16-byte load; 4 lanes make one 32-slot word
+    // 8 buckets per 16-byte load; 4 lanes make one 32-slot word.  Two codes
+    // (< 2^15) are compared per 32-bit add: code + (0x8000 - bstar - 1) has
+    // bit 15 of its halfword set exactly when code > bstar, and no carry
+    // reaches the other halfword.  The vectors holding slots outside
+    // [first, cand) (at most the first and the last) are tested one slot at
+    // a time, since codes past the last candidate were never written.
     const int nq = (cand + 7) / 8;
+    const uint32_t k_gt = (uint32_t)(0x8000 - bstar - 1) * 0x00010001u;
+    const uint32_t k_ge = (uint32_t)(0x8000 - bstar) * 0x00010001u;
     for (int q0 = warp * 32; q0 < nq; q0 += (NT / 32) * 32) {
         const int q = q0 + lane;
         uint32_t m = 0u;
         if (q < nq) {
             const uint4 c4 = *reinterpret_cast<const uint4*>(&o.code[8 * q]);
             const uint32_t cw[4] = {c4.x, c4.y, c4.z, c4.w};
+            uint32_t eq = 0u;
+            if (8 * q >= first && 8 * q + 8 <= cand) {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int t = 8 * q + i;
-                const int b = (int)((cw[i >> 1] >> (16 * (i & 1))) & 0xffffu);
-                if (t < cand && t >= first) {
-                    if (b > bstar) m |= 1u << i;
-                    else if (b == bstar) {
-                        const int pos = atomicAdd(&sm.n_list, 1);
-                        if (pos < kOneListCap) o.list_slot[pos] = t;
+                for (int j = 0; j < 4; ++j) {
+                    const uint32_t g = (cw[j] + k_gt) & 0x80008000u;
+                    const uint32_t e = ((cw[j] + k_ge) & 0x80008000u) & ~g;
+                    m |= ((g >> 15) & 1u) << (2 * j) | (g >> 31) << (2 * j + 1);
+                    eq |= ((e >> 15) & 1u) << (2 * j) | (e >> 31) << (2 * j + 1);
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int t = 8 * q + i;
+                    const int b = (int)((cw[i >> 1] >> (16 * (i & 1))) & 0xffffu);
+                    if (t < cand && t >= first) {
+                        if (b > bstar) m |= 1u << i;
+                        else if (b == bstar) eq |= 1u << i;
                     }
                 }
+            }
+            for (; eq; eq &= eq - 1u) {
+                const int pos = atomicAdd(&sm.n_list, 1);
+                if (pos < kOneListCap) o.list_slot[pos] = 8 * q + (__ffs(eq) - 1);
             }
         }
         uint32_t word = m << (8 * (lane & 3));
@@ -506,8 +554,8 @@ __device__ bool select_linear(const float* __restrict__ sc, int cand, int first,
         for (int j = threadIdx.x; j < take; j += NT) sidx[j] = first + j;
         return true;
     }
+    if (cand <= kCodeSlots) return select_one_pass<NT>(sc, cand, first, take, lo, span, sidx, sm);
     const float scale = (float)(kLinBins - 1) / span;
-    if (cand <= kCodeSlots) return select_one_pass<NT>(sc, cand, first, take, lo, scale, sidx, sm);
     int* hist = sm.u.sel.hist;
     // warp segments of whole 128-slot steps
     const int seg = ((cand + (NT / 32) - 1) / (NT / 32) + kStep - 1) / kStep * kStep;
