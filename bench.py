@@ -687,10 +687,13 @@ def run_decode(args, world, rank, local, dist, cfg):
         wl.cur_pos += cfg.decode_append
         lens = wl.seq_len.tolist()
         free_before = int(fl.count.item())
-        flush()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         pev = [torch.cuda.Event(enable_timing=True) for _ in range(4)] if args.phases else None
         torch.cuda.synchronize(dev)
+        # the flush keeps the GPU busy while the host enqueues the step, as
+        # in a decode loop whose host runs ahead of the GPU; without it the
+        # round's events would also time the host's launch of the step
+        flush()
         a.record()
         tri.tri_compress_step_ex(cache, qbar, qabs, R, cfg.base, wl.deltas, opt, ws, free_list=fl, idx_out=idx,
                                  events=pev)
