@@ -25,6 +25,7 @@ namespace {
 constexpr int kTableThreads = 256;
 constexpr int kDistThreads = 256;
 constexpr int kDistChunk = 4096;        // slots per score CTA
+constexpr int kDistVecs = 4;            // 4-slot vectors per thread whose reads are in flight together
 
 // Block (lh, chunk): coefficients of (l, h) in shared memory, then one table
 // entry per thread.
@@ -121,20 +122,60 @@ __global__ void __launch_bounds__(kDistThreads) distance_score_kernel(const Dist
         hi = max(hi, key);
         return v;
     };
-    // Four slots per thread and step: one 16-byte position load, four
-    // independent table reads, one 16-byte score store (t0 and the unit rows
-    // are multiples of 4 slots, so both accesses are aligned).
+    // 16-byte position loads and score stores (t0 and the unit rows are
+    // multiples of 4 slots, so both are aligned).
     const int n4 = (t1 - t0) >> 2;
     const int4* pos4 = reinterpret_cast<const int4*>(pos + t0);
     float4* out4 = reinterpret_cast<float4*>(out + t0);
-    for (int i = threadIdx.x; i < n4; i += kDistThreads) {
-        const int4 q = pos4[i];
-        float4 v;
-        v.x = score_one(q.x);
-        v.y = score_one(q.y);
-        v.z = score_one(q.z);
-        v.w = score_one(q.w);
-        out4[i] = v;
+    if (P >= 0 && P <= 0x7fffffff) {
+        // The usual case.  The lookup is two dependent reads per slot, so a
+        // thread first issues all its position loads (kDistVecs x 4 slots),
+        // then all their table reads, and the distance is formed in 32 bits:
+        // P - pos as an unsigned number is in range exactly when 0 <= d <=
+        // max_dist (a position after P wraps to a large value).
+        const uint32_t Pu = (uint32_t)P, maxd = (uint32_t)p.max_dist;
+        for (int i0 = threadIdx.x; i0 < n4; i0 += kDistThreads * kDistVecs) {
+            int4 q[kDistVecs];
+#pragma unroll
+            for (int k = 0; k < kDistVecs; ++k) {
+                const int i = i0 + k * kDistThreads;
+                q[k] = i < n4 ? __ldcs(pos4 + i) : make_int4((int)Pu, (int)Pu, (int)Pu, (int)Pu);
+            }
+            float v[kDistVecs][4];
+#pragma unroll
+            for (int k = 0; k < kDistVecs; ++k) {
+                const int32_t qc[4] = {q[k].x, q[k].y, q[k].z, q[k].w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const uint32_t d = Pu - (uint32_t)qc[c];
+                    bad |= d > maxd;
+                    v[k][c] = __ldg(tab + min(d, maxd));
+                }
+            }
+#pragma unroll
+            for (int k = 0; k < kDistVecs; ++k) {
+                const int i = i0 + k * kDistThreads;
+                if (i < n4) {
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t key = order_key(v[k][c]);
+                        lo = min(lo, key);
+                        hi = max(hi, key);
+                    }
+                    out4[i] = make_float4(v[k][0], v[k][1], v[k][2], v[k][3]);
+                }
+            }
+        }
+    } else {
+        for (int i = threadIdx.x; i < n4; i += kDistThreads) {
+            const int4 q = pos4[i];
+            float4 v;
+            v.x = score_one(q.x);
+            v.y = score_one(q.y);
+            v.z = score_one(q.z);
+            v.w = score_one(q.w);
+            out4[i] = v;
+        }
     }
     for (int t = t0 + 4 * n4 + threadIdx.x; t < t1; t += kDistThreads) out[t] = score_one(pos[t]);
     if (__syncthreads_or(bad) && threadIdx.x == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
