@@ -304,8 +304,8 @@ __device__ __forceinline__ int lin_bucket(float x, float lo, float scale, int nb
 
 // Emit the set bits of `bits` (nwords words, slot 32w + b) into sidx in
 // ascending order, at most `take` of them.  Each warp takes a contiguous run
-// of words.  A dense run (more than a quarter of its bits set) is walked a
-// word per step, lane i testing bit i, so every lane stores at once; a
+// of words.  A dense run (more than a quarter of its bits set) is walked
+// four words per step, lane i testing bit i, so every lane stores at once; a
 // sparse run is walked 64 words per step, lane i owning words 2i and 2i + 1:
 // a warp scan of their bit counts gives each lane its first output slot and
 // the lane stores its own set bits in order.
@@ -322,12 +322,18 @@ __device__ void emit_kept(const uint32_t* bits, int nwords, int take, int* sidx,
     int base = 0;
     for (int k = 0; k < warp; ++k) base += sm.warp_a[k];
     if (4 * cnt > 32 * (w1 - w0)) {
+        // four words per step: their loads do not wait on the running count
         const uint32_t lt = lanemask_lt();
-        for (int w = w0; w < w1; ++w) {
-            const uint32_t kw = bits[w];
-            const int pos = base + __popc(kw & lt);
-            if (((kw >> lane) & 1u) && pos < take) sidx[pos] = w * 32 + lane;
-            base += __popc(kw);
+        for (int w = w0; w < w1; w += 4) {
+            uint32_t kw[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) kw[i] = w + i < w1 ? bits[w + i] : 0u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int pos = base + __popc(kw[i] & lt);
+                if (((kw[i] >> lane) & 1u) && pos < take) sidx[pos] = (w + i) * 32 + lane;
+                base += __popc(kw[i]);
+            }
         }
     } else {
         for (int c0 = w0; c0 < w1; c0 += 64) {
