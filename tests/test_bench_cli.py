@@ -160,3 +160,19 @@ def test_gpus_flag_with_sequence_sharding_is_weak_scaling():
 def test_world_size_must_match_gpus_flag():
     r = _run(["--gpus", "4", "--steps", "1"], env_extra={"WORLD_SIZE": "2", "RANK": "0", "LOCAL_RANK": "0"})
     assert r.returncode != 0 and "WORLD_SIZE=2" in (r.stderr + r.stdout)
+
+
+def test_launch_accounting_and_flush_options():
+    """The launch count the bench line claims and the kernels it names follow
+    the step's shape: three launches when the step selects and compacts in
+    one persistent kernel, five with the separate kernels, for either score
+    mode; the L2 flush mode is a choice between two documented options."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.launches_per_step(True) == 3
+    assert bench.launches_per_step(False) == 5
+    assert bench.kernel_list(True, False) == "query_kernel, score kernel, select_compact_kernel"
+    assert bench.kernel_list(True, True) == "query_kernel (plan only), distance_score_kernel, select_compact_kernel"
+    assert bench.kernel_list(False, False).endswith("evict_kernel, move_kernel x2")
+    assert bench.parse_args([]).l2_flush == "clean"
+    assert bench.parse_args(["--l2-flush", "dirty"]).l2_flush == "dirty"
