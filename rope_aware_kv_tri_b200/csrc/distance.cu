@@ -89,24 +89,41 @@ __global__ void __launch_bounds__(kTableThreads) distance_table_kernel(const Dis
 
 // Block (u, chunk): slots [chunk*kDistChunk, ...) of unit u.
 __global__ void __launch_bounds__(kDistThreads) distance_score_kernel(const DistScoreParams p) {
+    static_assert(kDistChunk == kDistThreads * kDistVecs * 4, "one batch of position loads per CTA");
     __shared__ uint32_t wlo[kDistThreads / 32], whi[kDistThreads / 32];
     allow_next_grid();
-    wait_prior_grid();
     const int u = blockIdx.x;
     const int LH = p.L * p.Hkv;
     const int s = u / LH, lh = u % LH;
+    const int t0 = blockIdx.y * kDistChunk;
+    // The query position and this chunk's slot positions are inputs the plan
+    // does not write (the previous step's compaction wrote them before the
+    // plan began), so they are requested before waiting for the plan, up to
+    // the caller's length of the sequence (the plan validates it after).
+    const int64_t P = p.cur_pos[s];
+    const int32_t* pos = p.slot_pos + (int64_t)u * p.pos_stride;
+    const int4* pos4 = reinterpret_cast<const int4*>(pos + t0);
+    int n4_pre = 0;
+    if (p.seq_len_in) {
+        const int64_t n_in = min((int64_t)__ldg(p.seq_len_in + s), p.pos_stride) - t0;
+        n4_pre = n_in > 0 ? (int)(min(n_in, (int64_t)kDistChunk) >> 2) : 0;
+    }
+    int4 q[kDistVecs];
+#pragma unroll
+    for (int k = 0; k < kDistVecs; ++k) {
+        const int i = threadIdx.x + k * kDistThreads;
+        q[k] = i < n4_pre ? __ldcs(pos4 + i) : make_int4(0, 0, 0, 0);
+    }
+    wait_prior_grid();
     const int len = p.lens[s];
     if (len < 0 || (int64_t)len > p.pos_stride) {
         if (threadIdx.x == 0 && blockIdx.y == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
         return;
     }
     if (len <= p.trigger) return;            // a sequence the step leaves alone
-    const int t0 = blockIdx.y * kDistChunk;
     if (t0 >= len) return;
     const int t1 = min(t0 + kDistChunk, len);
-    const int64_t P = p.cur_pos[s];
     const float* tab = p.table + (int64_t)lh * (p.max_dist + 1);
-    const int32_t* pos = p.slot_pos + (int64_t)u * p.pos_stride;
     float* out = p.scores + (int64_t)u * p.score_stride;
     uint32_t lo = 0xffffffffu, hi = 0u;
     bool bad = false;
@@ -125,21 +142,21 @@ __global__ void __launch_bounds__(kDistThreads) distance_score_kernel(const Dist
     // 16-byte position loads and score stores (t0 and the unit rows are
     // multiples of 4 slots, so both are aligned).
     const int n4 = (t1 - t0) >> 2;
-    const int4* pos4 = reinterpret_cast<const int4*>(pos + t0);
     float4* out4 = reinterpret_cast<float4*>(out + t0);
     if (P >= 0 && P <= 0x7fffffff) {
         // The usual case.  The lookup is two dependent reads per slot, so a
-        // thread first issues all its position loads (kDistVecs x 4 slots),
+        // thread has all its position loads (kDistVecs x 4 slots) in flight,
         // then all their table reads, and the distance is formed in 32 bits:
         // P - pos as an unsigned number is in range exactly when 0 <= d <=
         // max_dist (a position after P wraps to a large value).
         const uint32_t Pu = (uint32_t)P, maxd = (uint32_t)p.max_dist;
-        for (int i0 = threadIdx.x; i0 < n4; i0 += kDistThreads * kDistVecs) {
-            int4 q[kDistVecs];
+        {
+            const int i0 = threadIdx.x;
 #pragma unroll
             for (int k = 0; k < kDistVecs; ++k) {
                 const int i = i0 + k * kDistThreads;
-                q[k] = i < n4 ? __ldcs(pos4 + i) : make_int4((int)Pu, (int)Pu, (int)Pu, (int)Pu);
+                if (i >= n4) q[k] = make_int4((int)Pu, (int)Pu, (int)Pu, (int)Pu);
+                else if (i >= n4_pre) q[k] = __ldcs(pos4 + i);    // past the caller's length: not prefetched
             }
             float v[kDistVecs][4];
 #pragma unroll

@@ -392,6 +392,7 @@ DistScoreParams make_distance_params(const tri_kv_desc* desc, const float* table
     d.pos_stride = (int64_t)desc->max_blocks * kBlockRows;
     d.cur_pos = desc->cur_pos;
     d.lens = desc->seq_len;
+    d.seq_len_in = desc->seq_len;
     d.trigger = -1;
     d.scores = scores;
     d.score_stride = (int64_t)desc->max_blocks * kBlockRows;

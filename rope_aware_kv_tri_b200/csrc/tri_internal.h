@@ -230,7 +230,8 @@ struct DistScoreParams {
     const int32_t* slot_pos;  // [U][pos_stride]
     int64_t pos_stride;       // max_blocks * 16
     const int64_t* cur_pos;
-    const int32_t* lens;      // [S]
+    const int32_t* lens;      // [S] lengths the step works from (the plan's validated copy)
+    const int32_t* seq_len_in; // [S] the caller's lengths (read before the plan completes; bounds prefetches only)
     int trigger;              // units of sequences with len <= trigger are skipped (-1: none)
     float* scores;
     int64_t score_stride;
