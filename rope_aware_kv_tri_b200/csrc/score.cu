@@ -151,21 +151,37 @@ __device__ void produce(const ScoreParams& p, uint8_t* tiles, uint64_t* full, ui
     const uint32_t stages = (uint32_t)p.stages;
     const uint32_t stage_bytes = (uint32_t)HG * kTileBytes;
     const int n_hg = p.Hkv / HG;
-    const int total = p.item_off[p.S];
     const uint64_t pol = l2_policy_evict_first();
+    // The work items, by the plan's rule, from inputs the plan does not
+    // write (the caller's lengths, the trigger, the statistics veto): the
+    // producer needs nothing from the plan, so it streams keys while the
+    // plan and the effective queries are still being built.  A length out
+    // of range counts as empty (the plan flags it).
+    const int64_t max_len = (int64_t)p.max_blocks * kBlockRows;
+    const bool vetoed = p.abort_word != nullptr && *reinterpret_cast<const volatile int32_t*>(p.abort_word) != 0;
+    auto seq_items = [&](int s, int& len) -> int {
+        int n = __ldg(p.seq_len_in + s);
+        if (n < 0 || (int64_t)n > max_len) n = 0;
+        len = n;
+        const bool scored = !vetoed && (p.budget <= 0 || n > p.trigger);
+        const int nblk = (n + kBlockRows - 1) / kBlockRows;
+        return scored ? p.L * n_hg * ((nblk + kChunkBlocks - 1) / kChunkBlocks) : 0;
+    };
+    int cs = 0, base = 0, len = 0;               // sequence cs holds items [base, base + cnt)
+    int cnt = p.S > 0 ? seq_items(0, len) : 0;
     uint32_t k = 0;
     bool ok = true;
-    for (int item = blockIdx.x; ok && item < total; item += gridDim.x) {
-        int lo = 0, hi = p.S;                    // item_off[lo] <= item < item_off[hi]
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (p.item_off[mid] <= item) lo = mid; else hi = mid;
+    for (int item = blockIdx.x; ok; item += gridDim.x) {
+        while (cs < p.S && item >= base + cnt) {
+            base += cnt;
+            ++cs;
+            cnt = cs < p.S ? seq_items(cs, len) : 0;
         }
-        const int s = lo;
-        const int len = p.len_ws[s];
+        if (cs >= p.S) break;
+        const int s = cs;
         const int nblk = (len + kBlockRows - 1) / kBlockRows;
         const int nch = (nblk + kChunkBlocks - 1) / kChunkBlocks;
-        const int r = item - p.item_off[s];
+        const int r = item - base;
         const int chunk = r % nch, lhg = r / nch;
         const int hg = lhg % n_hg, l = lhg / n_hg;
         const int unit0 = (s * p.L + l) * p.Hkv + hg * HG;
@@ -406,12 +422,13 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_kernel(const ScorePara
     }
     __syncthreads();
     allow_next_grid();
-    wait_prior_grid();          // the folded queries and the plan come from query_kernel
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (warp == kConsumerWarps) {
+        // plans its own work items: starts streaming before query_kernel ends
         if (lane == 0) produce(p, tiles, full, empty, meta, abort_flag);
         return;
     }
+    wait_prior_grid();          // the folded queries come from query_kernel
     if constexpr (AGG == 0)
         consume(p, warp, lane, tiles, full, empty, meta, abort_flag);
     else

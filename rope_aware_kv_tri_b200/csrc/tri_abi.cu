@@ -210,6 +210,7 @@ ScoreParams make_score_params(const tri_kv_desc* d, const uint8_t* ws, const WsL
     s.max_blocks = d->max_blocks;
     s.heads_per_tile = score_heads_per_tile(d->Hkv);
     s.agg_heads = 0;
+    s.seq_len_in = d->seq_len;
     return s;
 }
 
@@ -613,6 +614,9 @@ tri_status tri_compress_step_ex(tri_kv_desc* desc, const float* qbar, const floa
     float* scores = reinterpret_cast<float*>(ws + w.scores);
     ScoreParams sp = make_score_params(desc, ws, w, scores, (int64_t)desc->max_blocks * kBlockRows);
     sp.agg_heads = per_head ? desc->G : 0;
+    sp.budget = budget;
+    sp.trigger = trigger;
+    sp.abort_word = veto;
     if ((st = cuda_status(launch_score(sp, max_score_items(desc), device_sm_count(), stream, pdl))) != TRI_OK)
         return st;
     if (events) record(events->after_score, stream);

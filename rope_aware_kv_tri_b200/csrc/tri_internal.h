@@ -90,6 +90,12 @@ struct ScoreParams {
     int agg_heads;            // 0: folded group mean; G: max over G per-head scores
     int cuda_cores_only;      // 1: never the tensor-core max kernel
     int stages;
+    // The CUDA-core kernel's producer plans its own work items from these,
+    // by the plan's rule, so that it can stream keys before the plan ends.
+    const int32_t* seq_len_in; // [S] the caller's lengths
+    int budget;                // > 0: only sequences longer than `trigger` are scored
+    int trigger;
+    const int32_t* abort_word; // non-zero: the step was vetoed (nothing scored), or null
 };
 int score_heads_per_tile(int Hkv);
 cudaError_t launch_score(const ScoreParams& p, int max_items, int num_sms, cudaStream_t stream, bool pdl = false);
