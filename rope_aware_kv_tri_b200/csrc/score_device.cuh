@@ -1,6 +1,5 @@
-// score_device.cuh - the per-key score of the mean-aggregated path, shared
-// by the score kernel (score.cu) and the fused step kernel (step_fused.cu) so
-// both compute every score with the same instructions in the same order.
+// score_device.cuh - the per-key score of the mean-aggregated path and the
+// coefficient loads it needs (used by the score kernel, score.cu).
 //
 // Pages: "TriAttention: Trigonometric KV Compression for Efficient Long
 // Reasoning" - "Key Concepts", Trigonometric Distance Preference and Norm as
