@@ -68,7 +68,9 @@ template <int G>
 struct MmaShape {
     static constexpr int N = 8 * 2 * G;                       // accumulator columns
     static constexpr uint32_t kCBytes = N * 256;              // C: two halves of N rows x 128 B
-    static constexpr uint32_t kWBytes = 8 * G * 64 * 4;       // norm weights of 8 units
+    static constexpr int kWHead = G * 64 + 4;                 // floats per unit: padded by 16 bytes so that
+                                                              // the two units a warp reads sit in other banks
+    static constexpr uint32_t kWBytes = 8 * kWHead * 4;       // norm weights of 8 units
     static constexpr uint32_t kAccCols = kGroups * N;         // one accumulator per epilogue group
     static constexpr uint32_t kTmemCols = kAccCols <= 32 ? 32 : kAccCols <= 64 ? 64 : kAccCols <= 128 ? 128
                                         : kAccCols <= 256 ? 256 : 512;
@@ -391,7 +393,10 @@ __device__ void write_coefficients(const ScoreParams& p, int unit0, uint8_t* C, 
 #pragma unroll
         for (int i = 0; i < kWBatch; ++i) wv[i] = __ldg(wsrc + lane + 32 * (i0 + i));
 #pragma unroll
-        for (int i = 0; i < kWBatch; ++i) wdst[lane + 32 * (i0 + i)] = wv[i];
+        for (int i = 0; i < kWBatch; ++i) {
+            const int f = lane + 32 * (i0 + i);                 // float4 of unit f / (G * 16)
+            wdst[f + f / (G * 16)] = wv[i];
+        }
     }
 }
 
@@ -535,7 +540,7 @@ __device__ void mma_epilogue(const ScoreParams& p, const Smem& sm, uint32_t tmem
             }
             // band magnitudes of the key, weighted per head
             const uint8_t* st = sm.stages + (size_t)slot * kStageBytes;
-            const float* W = sm.wbuf + (size_t)(m.ord & 1) * (Sh::kWBytes / 4) + (size_t)hh * G * kBands;
+            const float* W = sm.wbuf + (size_t)(m.ord & 1) * (Sh::kWBytes / 4) + (size_t)hh * Sh::kWHead;
             float2 wn[G];
 #pragma unroll
             for (int g = 0; g < G; ++g) wn[g] = make_float2(0.f, 0.f);
