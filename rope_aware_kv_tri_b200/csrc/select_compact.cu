@@ -19,13 +19,20 @@
 //  * selects its kept slots (select_device.cuh), writes its indices, and
 //    carries slot positions with the rows when asked (distance-table step);
 //  * packs the at-risk prefix [m0, J) in place in ordered rounds (rows whose
-//    sources a later store overwrites);
+//    sources a later store overwrites): each round has the TMA engine copy
+//    up to 192 rows (one row's K and V per thread, 256-byte bulk copies
+//    counted on one mbarrier) into the (now idle) selection scratch, then
+//    stores them with bulk stores;
 //  * moves rows [J, kept): their sources idx_j >= kept are never written in
 //    the step, and the prefix pass has read every destination row it needed.
-//    Each warp takes rows J + 32w, J + 32(w + 16), ... and moves them 12 at
-//    a time through its own slice of the (now idle) selection scratch with
-//    16-byte asynchronous copies (lanes 0-15 the K half of a row, 16-31 the V
-//    half): 96 KiB in flight per CTA;
+//    Each warp takes rows J + w, J + w + 16, ... and moves them 12 at a time
+//    through its own 6 KiB of the scratch, with bulk copies counted on its
+//    own mbarrier: 96 KiB in flight per CTA.
+//    Bulk copies move a row with two instructions where 16-byte copies take
+//    32 loads and 32 stores: the rounds and moves run closer to the copy
+//    bandwidth (one 32-layer x 8-head step of 32768 keys per unit keeping
+//    2048: 127 -> 117 us; a decode round of 16 sequences keeping 2048 of
+//    2176 slots: 1.93 -> 1.76 ms);
 //  * does its sequence's bookkeeping (new length, freed blocks; first head
 //    of layer 0).
 //
@@ -52,7 +59,11 @@ constexpr int kRowPairBytes = 2 * kHeadDim * 2;    // a K row and a V row: 512 b
 using ScSmem = EvictSmem<kScThreads>;
 
 __host__ __device__ inline size_t sc_sidx_offset() { return (sizeof(ScSmem) + 15) / 16 * 16; }
-__host__ __device__ inline size_t sc_smem_bytes(int budget) { return sc_sidx_offset() + (size_t)budget * 4; }
+// the mbarriers after the kept indices: one for the prefix rounds, one per warp for the moves
+__host__ __device__ inline size_t sc_bar_offset(int budget) {
+    return (sc_sidx_offset() + (size_t)budget * 4 + 7) / 8 * 8;
+}
+__host__ __device__ inline size_t sc_smem_bytes(int budget) { return sc_bar_offset(budget) + 8 * (1 + kScWarps); }
 
 static_assert(sizeof(SelectScratch) >= (size_t)kScWarps * kScMoveRows * kRowPairBytes,
               "move staging must fit in the selection scratch");
@@ -61,25 +72,27 @@ __device__ __forceinline__ bool compressed(const SelectCompactParams& p, int u) 
     return __ldcg(p.len_ws + u / (p.L * p.Hkv)) > p.trigger;
 }
 
-// Rows [J, kept) of unit u take their sources idx_j (>= kept).  Warp w
-// takes rows J + 32w + 512k; lane i resolves one row of the 32, then the
-// warp copies its rows kScMoveRows at a time through its 6 KiB staging slice.
+// Rows [J, kept) of unit u take their sources idx_j (>= kept), which no store
+// of the step touches, so they move in any order: warp w takes rows J + w,
+// J + w + 16, ..., kScMoveRows at a time; lane i of a batch has the TMA engine
+// copy its row's K and V (256 bytes each) into the warp's 6 KiB of the idle
+// selection scratch, counted on the warp's mbarrier, then stores them with
+// bulk stores and waits until those have read the staging.
 __device__ void move_rows(const SelectCompactParams& p, int u, int s, int l, int h, int len, int J, const int* sidx,
-                          uint8_t* stage) {
+                          uint8_t* stage, uint64_t* wbar, uint32_t& wphase) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = p.budget;
     const int32_t* bt = p.block_table + (int64_t)s * p.max_blocks;
     const int64_t lt = (int64_t)l * p.num_blocks;
-    uint8_t* wbuf = stage + (size_t)warp * kScMoveRows * kRowPairBytes;
-    const int half = lane < 16 ? 0 : kHeadDim * 2;     // K or V half of the staged row pair
-    const int in_row = (lane & 15) * 16;
-    uint8_t* pool = lane < 16 ? p.k_pool : p.v_pool;
+    uint8_t* mine = stage + ((size_t)warp * kScMoveRows + lane) * kRowPairBytes;
+    uint64_t* bar = wbar + warp;
+    const uint64_t pol = l2_policy_evict_first();
     bool bad = false;
-    for (int j0 = J + warp * 32; j0 < B; j0 += kScThreads) {
-        const int j = j0 + lane;
+    for (int j0 = J + warp; j0 < B; j0 += kScWarps * kScMoveRows) {
+        const int j = j0 + lane * kScWarps;
         int64_t so = 0, dof = 0;
         bool valid = false;
-        if (j < B) {
+        if (lane < kScMoveRows && j < B) {
             const int src = sidx[j];
             if (src >= B && src < len) {
                 if (row_offset(bt, src, lt, p.Hkv, h, p.num_blocks, so) &&
@@ -89,30 +102,89 @@ __device__ void move_rows(const SelectCompactParams& p, int u, int s, int l, int
                     bad = true;
             }
         }
-        uint32_t todo = __ballot_sync(0xffffffffu, valid);
-        while (todo) {
-            uint32_t batch = todo;
-            if (__popc(todo) > kScMoveRows) batch = todo & ((1u << __fns(todo, 0, kScMoveRows + 1)) - 1u);
-            int n = 0;
-            for (uint32_t b = batch; b; b &= b - 1u, ++n) {
-                const long long src_off = __shfl_sync(0xffffffffu, (long long)so, __ffs(b) - 1);
-                cp_async16(wbuf + n * kRowPairBytes + half + in_row, pool + src_off + in_row);
-            }
-            cp_async_wait_all();
-            n = 0;
-            for (uint32_t b = batch; b; b &= b - 1u, ++n) {
-                const long long dst_off = __shfl_sync(0xffffffffu, (long long)dof, __ffs(b) - 1);
-                *reinterpret_cast<uint4*>(pool + dst_off + in_row) =
-                    *reinterpret_cast<const uint4*>(wbuf + n * kRowPairBytes + half + in_row);
-            }
-            todo &= ~batch;
+        const uint32_t nvalid = __popc(__ballot_sync(0xffffffffu, valid));
+        if (lane == 0) mbar_arrive_expect_tx(bar, nvalid * kRowPairBytes);
+        if (valid) {
+            bulk_copy_g2s(mine, p.k_pool + so, kRowPairBytes / 2, bar, pol);
+            bulk_copy_g2s(mine + kRowPairBytes / 2, p.v_pool + so, kRowPairBytes / 2, bar, pol);
         }
+        const bool landed = mbar_wait_bounded(bar, wphase);
+        if (!landed) {
+            if (lane == 0) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
+            mbar_wait_bounded(bar, wphase);
+            wphase ^= 1u;
+            break;
+        }
+        wphase ^= 1u;
+        if (valid) {
+            bulk_copy_s2g(p.k_pool + dof, mine, kRowPairBytes / 2);
+            bulk_copy_s2g(p.v_pool + dof, mine + kRowPairBytes / 2, kRowPairBytes / 2);
+            bulk_commit_group();
+            bulk_wait_group_read<0>();
+        }
+        __syncwarp();
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
 }
 
+// The at-risk prefix [m0, J) in ascending rounds of kStageRows rows staged in
+// the idle selection scratch: thread i of a round has the TMA engine copy row
+// base + i's source (its K and V rows, 256 bytes each) into shared memory,
+// every copy of the round counted on one mbarrier; then each thread has the
+// staged rows stored to their destinations with bulk stores and waits until
+// those have read the staging.  A later round reads only slots >= its first
+// row, which no earlier round writes.
+__device__ bool pack_prefix_bulk(const SelectCompactParams& p, const int* sidx, int m0, int J, int s, int l, int h,
+                                 uint8_t* stage, uint64_t* bar, uint32_t& phase) {
+    const int tid = threadIdx.x;
+    const int32_t* bt = p.block_table + (int64_t)s * p.max_blocks;
+    const int64_t lt = (int64_t)l * p.num_blocks;
+    const uint64_t pol = l2_policy_evict_first();
+    bool bad = false;
+    fence_proxy_async_smem();           // the selection's stores to the scratch precede the copies into it
+    sel_sync<kScThreads>();
+    for (int base = m0; base < J; base += kStageRows) {
+        const int n = min(kStageRows, J - base);
+        int64_t so = 0, dof = 0;
+        bool valid = false;
+        if (tid < n) {
+            const int j = base + tid;
+            if (row_offset(bt, sidx[j], lt, p.Hkv, h, p.num_blocks, so) &&
+                row_offset(bt, j, lt, p.Hkv, h, p.num_blocks, dof))
+                valid = true;
+            else
+                bad = true;
+        }
+        const int nvalid = __syncthreads_count(valid);
+        if (tid == 0) mbar_arrive_expect_tx(bar, (uint32_t)nvalid * kRowPairBytes);
+        uint8_t* mine = stage + (size_t)tid * kRowPairBytes;
+        if (valid) {
+            bulk_copy_g2s(mine, p.k_pool + so, kRowPairBytes / 2, bar, pol);
+            bulk_copy_g2s(mine + kRowPairBytes / 2, p.v_pool + so, kRowPairBytes / 2, bar, pol);
+        }
+        if (!mbar_wait_bounded(bar, phase)) {
+            // the copies did not land in time: flag it, let them land (bounded), store nothing
+            if (tid == 0) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
+            mbar_wait_bounded(bar, phase);
+            phase ^= 1u;
+            sel_sync<kScThreads>();
+            return bad;
+        }
+        phase ^= 1u;
+        if (valid) {
+            bulk_copy_s2g(p.k_pool + dof, mine, kRowPairBytes / 2);
+            bulk_copy_s2g(p.v_pool + dof, mine + kRowPairBytes / 2, kRowPairBytes / 2);
+            bulk_commit_group();
+            bulk_wait_group_read<0>();
+        }
+        sel_sync<kScThreads>();         // the staging is free for the next round
+    }
+    return bad;
+}
+
 // Select unit u, pack its at-risk prefix in place, move its other kept rows.
-__device__ void select_task(const SelectCompactParams& p, int u, ScSmem& sm, int* sidx) {
+__device__ void select_task(const SelectCompactParams& p, int u, ScSmem& sm, int* sidx, uint64_t* bar,
+                            uint32_t& phase, uint32_t& wphase) {
     const int tid = threadIdx.x;
     const int LH = p.L * p.Hkv;
     const int s = u / LH, rem = u % LH, l = rem / p.Hkv, h = rem % p.Hkv;
@@ -140,9 +212,14 @@ __device__ void select_task(const SelectCompactParams& p, int u, ScSmem& sm, int
     }
     const int m0 = block_sum<kScThreads>(fixed, sm);   // idx_j == j exactly for j < m0
     const int J = block_sum<kScThreads>(low, sm);      // idx_j < kept exactly for j < J
-    if (J > m0 && sel_sync_or<kScThreads>(pack_ordered_prefix<kScThreads>(sidx, m0, J, s, l, h, p, sm)) && tid == 0)
+    if (J > m0 &&
+        sel_sync_or<kScThreads>(pack_prefix_bulk(p, sidx, m0, J, s, l, h, reinterpret_cast<uint8_t*>(&sm.u), bar,
+                                                 phase)) &&
+        tid == 0)
         raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
-    move_rows(p, u, s, l, h, len, J, sidx, reinterpret_cast<uint8_t*>(&sm.u));
+    fence_proxy_async_smem();           // the selection's stores to the scratch precede the copies into it
+    sel_sync<kScThreads>();
+    move_rows(p, u, s, l, h, len, J, sidx, reinterpret_cast<uint8_t*>(&sm.u), bar + 1, wphase);
     if (l == 0 && h == 0) {
         // the sequence's new length and its freed blocks
         const int32_t* bt = p.block_table + (int64_t)s * p.max_blocks;
@@ -166,6 +243,13 @@ __global__ void __launch_bounds__(kScThreads, 2) select_compact_kernel(const __g
     ScSmem& sm = *reinterpret_cast<ScSmem*>(smem);
     int* sidx = reinterpret_cast<int*>(smem + sc_sidx_offset());
     __shared__ int s_task;
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + sc_bar_offset(p.budget));
+    if (threadIdx.x == 0) {
+        for (int i = 0; i <= kScWarps; ++i) mbar_init(&bar[i], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    uint32_t phase = 0, wphase = 0;
     wait_prior_grid();          // scores, key ranges, plan and the zeroed unit counter
     if (p.abort_word && __ldcg(p.abort_word) != 0) return;    // vetoed step: change nothing
     const int U = p.S * p.L * p.Hkv;
@@ -179,7 +263,7 @@ __global__ void __launch_bounds__(kScThreads, 2) select_compact_kernel(const __g
         const int u = s_task;
         __syncthreads();
         if (u >= U) break;
-        select_task(p, u, sm, sidx);
+        select_task(p, u, sm, sidx, bar, phase, wphase);
     }
 }
 
