@@ -77,8 +77,10 @@ __device__ __forceinline__ bool compressed(const SelectCompactParams& p, int u) 
 // J + w + 16, ..., kScMoveRows at a time; lane i of a batch has the TMA engine
 // copy its row's K and V (256 bytes each) into the warp's 6 KiB of the idle
 // selection scratch, counted on the warp's mbarrier, then stores them with
-// bulk stores and waits until those have read the staging.
-__device__ void move_rows(const SelectCompactParams& p, int u, int s, int l, int h, int len, int J, const int* sidx,
+// bulk stores and waits until those have read the staging.  Returns true
+// (for the whole warp) when a batch's copies did not land in time: the
+// warp then stores nothing more and the status word says so.
+__device__ bool move_rows(const SelectCompactParams& p, int u, int s, int l, int h, int len, int J, const int* sidx,
                           uint8_t* stage, uint64_t* wbar, uint32_t& wphase) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int B = p.budget;
@@ -87,7 +89,7 @@ __device__ void move_rows(const SelectCompactParams& p, int u, int s, int l, int
     uint8_t* mine = stage + ((size_t)warp * kScMoveRows + lane) * kRowPairBytes;
     uint64_t* bar = wbar + warp;
     const uint64_t pol = l2_policy_evict_first();
-    bool bad = false;
+    bool bad = false, gave_up = false;
     for (int j0 = J + warp; j0 < B; j0 += kScWarps * kScMoveRows) {
         const int j = j0 + lane * kScWarps;
         int64_t so = 0, dof = 0;
@@ -109,13 +111,13 @@ __device__ void move_rows(const SelectCompactParams& p, int u, int s, int l, int
             bulk_copy_g2s(mine + kRowPairBytes / 2, p.v_pool + so, kRowPairBytes / 2, bar, pol);
         }
         const bool landed = mbar_wait_bounded(bar, wphase);
-        if (!landed) {
+        if (!landed) mbar_wait_bounded(bar, wphase);   // copies still in flight land before the staging is reused
+        wphase ^= 1u;
+        if (!__all_sync(0xffffffffu, landed)) {
             if (lane == 0) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
-            mbar_wait_bounded(bar, wphase);
-            wphase ^= 1u;
+            gave_up = true;
             break;
         }
-        wphase ^= 1u;
         if (valid) {
             bulk_copy_s2g(p.k_pool + dof, mine, kRowPairBytes / 2);
             bulk_copy_s2g(p.v_pool + dof, mine + kRowPairBytes / 2, kRowPairBytes / 2);
@@ -125,6 +127,7 @@ __device__ void move_rows(const SelectCompactParams& p, int u, int s, int l, int
         __syncwarp();
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
+    return gave_up;
 }
 
 // The at-risk prefix [m0, J) in ascending rounds of kStageRows rows staged in
@@ -133,9 +136,11 @@ __device__ void move_rows(const SelectCompactParams& p, int u, int s, int l, int
 // every copy of the round counted on one mbarrier; then each thread has the
 // staged rows stored to their destinations with bulk stores and waits until
 // those have read the staging.  A later round reads only slots >= its first
-// row, which no earlier round writes.
+// row, which no earlier round writes.  gave_up (the same in every thread)
+// says a round's copies did not land in time; that round stores only the
+// rows that did land, no later round runs, and the status word says so.
 __device__ bool pack_prefix_bulk(const SelectCompactParams& p, const int* sidx, int m0, int J, int s, int l, int h,
-                                 uint8_t* stage, uint64_t* bar, uint32_t& phase) {
+                                 uint8_t* stage, uint64_t* bar, uint32_t& phase, bool& gave_up) {
     const int tid = threadIdx.x;
     const int32_t* bt = p.block_table + (int64_t)s * p.max_blocks;
     const int64_t lt = (int64_t)l * p.num_blocks;
@@ -162,28 +167,30 @@ __device__ bool pack_prefix_bulk(const SelectCompactParams& p, const int* sidx, 
             bulk_copy_g2s(mine, p.k_pool + so, kRowPairBytes / 2, bar, pol);
             bulk_copy_g2s(mine + kRowPairBytes / 2, p.v_pool + so, kRowPairBytes / 2, bar, pol);
         }
-        if (!mbar_wait_bounded(bar, phase)) {
-            // the copies did not land in time: flag it, let them land (bounded), store nothing
-            if (tid == 0) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
-            mbar_wait_bounded(bar, phase);
-            phase ^= 1u;
-            sel_sync<kScThreads>();
-            return bad;
+        const bool landed = mbar_wait_bounded(bar, phase);
+        if (!landed) {
+            raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
+            mbar_wait_bounded(bar, phase);  // copies still in flight land before the staging is reused
         }
         phase ^= 1u;
-        if (valid) {
+        if (valid && landed) {
             bulk_copy_s2g(p.k_pool + dof, mine, kRowPairBytes / 2);
             bulk_copy_s2g(p.v_pool + dof, mine + kRowPairBytes / 2, kRowPairBytes / 2);
             bulk_commit_group();
             bulk_wait_group_read<0>();
         }
-        sel_sync<kScThreads>();         // the staging is free for the next round
+        if (sel_sync_or<kScThreads>(!landed)) {   // the staging is free for the next round
+            gave_up = true;
+            break;
+        }
     }
     return bad;
 }
 
 // Select unit u, pack its at-risk prefix in place, move its other kept rows.
-__device__ void select_task(const SelectCompactParams& p, int u, ScSmem& sm, int* sidx, uint64_t* bar,
+// Returns true (in every thread) when a wait for copies gave up: the CTA then
+// takes no further unit.
+__device__ bool select_task(const SelectCompactParams& p, int u, ScSmem& sm, int* sidx, uint64_t* bar,
                             uint32_t& phase, uint32_t& wphase) {
     const int tid = threadIdx.x;
     const int LH = p.L * p.Hkv;
@@ -212,14 +219,15 @@ __device__ void select_task(const SelectCompactParams& p, int u, ScSmem& sm, int
     }
     const int m0 = block_sum<kScThreads>(fixed, sm);   // idx_j == j exactly for j < m0
     const int J = block_sum<kScThreads>(low, sm);      // idx_j < kept exactly for j < J
+    bool gave_up = false;
     if (J > m0 &&
         sel_sync_or<kScThreads>(pack_prefix_bulk(p, sidx, m0, J, s, l, h, reinterpret_cast<uint8_t*>(&sm.u), bar,
-                                                 phase)) &&
+                                                 phase, gave_up)) &&
         tid == 0)
         raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
     fence_proxy_async_smem();           // the selection's stores to the scratch precede the copies into it
     sel_sync<kScThreads>();
-    move_rows(p, u, s, l, h, len, J, sidx, reinterpret_cast<uint8_t*>(&sm.u), bar + 1, wphase);
+    if (!gave_up) gave_up = move_rows(p, u, s, l, h, len, J, sidx, reinterpret_cast<uint8_t*>(&sm.u), bar + 1, wphase);
     if (l == 0 && h == 0) {
         // the sequence's new length and its freed blocks
         const int32_t* bt = p.block_table + (int64_t)s * p.max_blocks;
@@ -235,7 +243,7 @@ __device__ void select_task(const SelectCompactParams& p, int u, ScSmem& sm, int
         }
         if (tid == 0) p.seq_len_out[s] = B;
     }
-    sel_sync<kScThreads>();                // the scratch is free for the next unit
+    return sel_sync_or<kScThreads>(gave_up);    // the scratch is free for the next unit
 }
 
 __global__ void __launch_bounds__(kScThreads, 2) select_compact_kernel(const __grid_constant__ SelectCompactParams p) {
@@ -263,7 +271,7 @@ __global__ void __launch_bounds__(kScThreads, 2) select_compact_kernel(const __g
         const int u = s_task;
         __syncthreads();
         if (u >= U) break;
-        select_task(p, u, sm, sidx, bar, phase, wphase);
+        if (select_task(p, u, sm, sidx, bar, phase, wphase)) break;
     }
 }
 
