@@ -41,6 +41,8 @@ namespace {
 constexpr int kEvictThreads = 512;
 constexpr int kMoveThreads = 256;
 constexpr int kMoveRows = 8;                      // rows in flight per warp in move_kernel
+constexpr int kMoveWarps = kMoveThreads / 32;
+constexpr size_t kMoveStageBytes = (size_t)kMoveWarps * kMoveRows * 2 * kRowBytes;   // 32 KiB
 using EvictSmemT = EvictSmem<kEvictThreads>;
 
 __global__ void __launch_bounds__(kEvictThreads, 2) evict_kernel(const EvictParams p) {
@@ -240,6 +242,13 @@ __device__ void copy_out_rows(const MoveParams& p) {
 }
 
 __global__ void __launch_bounds__(kMoveThreads, 3) move_kernel(const MoveParams p) {
+    extern __shared__ __align__(128) uint8_t move_smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(move_smem + kMoveStageBytes);   // one mbarrier per warp
+    if (threadIdx.x < kMoveWarps) {
+        mbar_init(&bars[threadIdx.x], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
     wait_prior_grid();
     if (p.abort_word && __ldcg(p.abort_word) != 0) return;    // vetoed step: move nothing
     if (p.copy_out) {
@@ -253,9 +262,13 @@ __global__ void __launch_bounds__(kMoveThreads, 3) move_kernel(const MoveParams 
     const int warp0 = (int)(((int64_t)blockIdx.x * kMoveThreads + threadIdx.x) >> 5);
     const int nwarps = (int)(((int64_t)gridDim.x * kMoveThreads) >> 5);
     const int64_t max_len = (int64_t)p.max_blocks * kBlockRows;
-    const int in_row = (lane & 15) * 16;
-    bool bad = false;
-    for (int tile = warp0; tile < ntiles; tile += nwarps) {
+    const int wl = threadIdx.x >> 5;
+    uint8_t* stage = move_smem + (size_t)wl * kMoveRows * 2 * kRowBytes;
+    uint64_t* bar = &bars[wl];
+    uint32_t phase = 0;
+    const uint64_t pol = l2_policy_evict_first();
+    bool bad = false, gave_up = false;
+    for (int tile = warp0; tile < ntiles && !gave_up; tile += nwarps) {
         const int u = tile / tiles_per_unit;
         const int j = (tile % tiles_per_unit) * 32 + lane;      // this lane's row
         const int s = u / LH, l = (u % LH) / p.Hkv, h = u % p.Hkv;
@@ -309,29 +322,36 @@ __global__ void __launch_bounds__(kMoveThreads, 3) move_kernel(const MoveParams 
                 }
             }
         }
+        // kMoveRows rows at a time: each row's lane has the TMA engine copy
+        // its K and V rows into the warp's staging (counted on the warp's
+        // mbarrier), then store them with bulk stores
         uint32_t todo = __ballot_sync(0xffffffffu, sk != nullptr);
         while (todo) {
-            uint4 buf[kMoveRows];
-            uint8_t* dst[kMoveRows];
-#pragma unroll
-            for (int k = 0; k < kMoveRows; ++k) {
-                const int r = todo ? __ffs(todo) - 1 : -1;
-                if (todo) todo &= todo - 1u;
-                const int rr = r < 0 ? 0 : r;
-                const unsigned long long s_k = __shfl_sync(0xffffffffu, (unsigned long long)sk, rr);
-                const unsigned long long s_v = __shfl_sync(0xffffffffu, (unsigned long long)sv, rr);
-                const unsigned long long d_k = __shfl_sync(0xffffffffu, (unsigned long long)dk, rr);
-                const unsigned long long d_v = __shfl_sync(0xffffffffu, (unsigned long long)dv, rr);
-                dst[k] = nullptr;
-                if (r >= 0) {
-                    const uint8_t* src = reinterpret_cast<const uint8_t*>(lane < 16 ? s_k : s_v);
-                    buf[k] = __ldcg(reinterpret_cast<const uint4*>(src + in_row));
-                    dst[k] = reinterpret_cast<uint8_t*>(lane < 16 ? d_k : d_v) + in_row;
-                }
+            uint32_t batch = todo;
+            if (__popc(todo) > kMoveRows) batch = todo & ((1u << __fns(todo, 0, kMoveRows + 1)) - 1u);
+            todo &= ~batch;
+            const bool in_batch = (batch >> lane) & 1u;
+            uint8_t* st = stage + (size_t)__popc(batch & ((1u << lane) - 1u)) * 2 * kRowBytes;
+            if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)__popc(batch) * 2 * kRowBytes);
+            if (in_batch) {
+                bulk_copy_g2s(st, sk, kRowBytes, bar, pol);
+                bulk_copy_g2s(st + kRowBytes, sv, kRowBytes, bar, pol);
             }
-#pragma unroll
-            for (int k = 0; k < kMoveRows; ++k)
-                if (dst[k]) *reinterpret_cast<uint4*>(dst[k]) = buf[k];
+            const bool landed = mbar_wait_bounded(bar, phase);
+            if (!landed) mbar_wait_bounded(bar, phase);   // copies still in flight land before the staging is reused
+            phase ^= 1u;
+            if (!__all_sync(0xffffffffu, landed)) {
+                if (lane == 0) raise_flag(p.status, TRI_DEVFLAG_TIMEOUT);
+                gave_up = true;
+                break;
+            }
+            if (in_batch) {
+                bulk_copy_s2g(dk, st, kRowBytes);
+                bulk_copy_s2g(dv, st + kRowBytes, kRowBytes);
+                bulk_commit_group();
+                bulk_wait_group_read<0>();
+            }
+            __syncwarp();
         }
     }
     if (__any_sync(0xffffffffu, bad) && lane == 0) raise_flag(p.status, TRI_DEVFLAG_BOUNDS);
@@ -466,7 +486,8 @@ cudaError_t launch_move(const MoveParams& p, int num_sms, cudaStream_t stream, b
     if (tiles > INT_MAX) return cudaErrorInvalidValue;
     int64_t grid = (tiles + kMoveThreads / 32 - 1) / (kMoveThreads / 32);
     if (grid > (int64_t)num_sms * 3) grid = (int64_t)num_sms * 3;
-    return launch_kernel(move_kernel, dim3((unsigned)grid), dim3(kMoveThreads), 0, stream, pdl, p);
+    const size_t smem = kMoveStageBytes + kMoveWarps * sizeof(uint64_t);
+    return launch_kernel(move_kernel, dim3((unsigned)grid), dim3(kMoveThreads), smem, stream, pdl, p);
 }
 
 cudaError_t launch_finalize(const FinalizeParams& p, cudaStream_t stream) {
